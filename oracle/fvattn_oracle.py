@@ -1,0 +1,385 @@
+"""CPU oracle for adaptive block-sparse spatiotemporal attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may use it.  It shares no code with the CUDA path; the
+only common module is the seeded input generator, which holds none of the
+method's arithmetic.
+
+Plain, slow and written to be checked by eye: numpy in float64, one step per
+function, in the order the pages give the method.  Library primitives
+(matmul, stable argsort, cumsum, exp) serve as steps; there is no blocking,
+fusion or reordering beyond the definitions below.
+
+Sources (page title, section):
+  * "VSA" digest (aibr.jp), section 3 "core technical elements": tokens are
+    grouped into small (4,4,4) cubes, a coarse stage pools each cube and
+    predicts per-tile importance, the fine stage runs token-level attention
+    only inside the selected tiles.
+  * "FVAttn" digest (iselia-ai.com), sections 00 and 02: the routing front end
+    is top-p routing with a top-k safety floor.
+  * "DFSAttn" digest (gist.science 2605.23445), section 1 "Hilbert shuffle":
+    tokens are reordered along a 3D Hilbert curve before blocking; section 3
+    "smart cache": the previous step's selection is reused.
+  * "Causal-RoPE SP" digest (gist.science 2603.06664), sections 2.2-2.3: 3D
+    rotary position encoding with precomputed frequencies.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * pooling is the mean over the 64 tokens of a tile;
+  * coarse logits are scale * Qp . Kp with scale = 1/sqrt(d); normalisation is
+    a softmax over the key tiles of each query-tile row;
+  * top-p keeps the fewest tiles (at least one) whose cumulative mass, summed
+    in descending order, reaches p (``>= p``); ties go to the lower tile
+    index; count = min(nT, max(m, k_min)); p >= 1 keeps every tile;
+  * the output is the fine stage only (the coarse stage only routes);
+  * lse is the natural log of the softmax normaliser;
+  * RoPE: per-axis groups of 44/42/42 head dims for (t, h, w), adjacent pairs
+    (2j, 2j+1) inside each group, angle = pos * base^(-2j/d_axis); pooling uses
+    the rotated values unrounded, the fine stage uses them rounded to bf16
+    (the tensor-core operand precision of a bf16 workload);
+  * Hilbert order: Skilling's transposed-axes Hilbert index ("Programming the
+    Hilbert curve", AIP Conf. Proc. 707, 2004) on the enclosing 2^k cube with
+    axes (t, h, w), valid tokens ordered by index.
+
+Every function below is pinned by ``tests/test_oracle_*.py`` against brute
+force, closed forms, invariants or library routines; see the pin list in the
+design notes.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+TILE = (4, 4, 4)
+
+
+# ----------------------------------------------------------------------------
+# token layout and the two orders
+# ----------------------------------------------------------------------------
+
+def token_coords(grid):
+    """(t, h, w) of every token in natural (raster) order, int64 [N, 3]."""
+    T, Hg, W = grid
+    n = np.arange(T * Hg * W, dtype=np.int64)
+    return np.stack([n // (Hg * W), (n // W) % Hg, n % W], axis=1)
+
+
+def check_grid(grid, tile=TILE):
+    for g, t in zip(grid, tile):
+        if g % t != 0:
+            raise ValueError(f"grid {grid} is not a multiple of the tile {tile}")
+
+
+def raster_cube_positions(grid, tile=TILE):
+    """Raster-cube order: position of each natural token in the tiled layout.
+
+    Tiles are ranked in raster order over the tile grid; inside a tile the
+    64 tokens are ranked in raster order of (t%4, h%4, w%4)."""
+    check_grid(grid, tile)
+    c = token_coords(grid)
+    nh, nw = grid[1] // tile[1], grid[2] // tile[2]
+    tile_rank = ((c[:, 0] // tile[0]) * nh + c[:, 1] // tile[1]) * nw + c[:, 2] // tile[2]
+    intra = ((c[:, 0] % tile[0]) * tile[1] + c[:, 1] % tile[1]) * tile[2] + c[:, 2] % tile[2]
+    return tile_rank * (tile[0] * tile[1] * tile[2]) + intra
+
+
+def hilbert_index_3d(coords, bits):
+    """Hilbert index of each 3D point (int64 [P, 3], each coordinate < 2^bits).
+
+    Skilling's method: convert the axes to the "transposed" Hilbert form
+    (undo the excess rotations from the top bit down, then Gray-encode), then
+    read the index out by interleaving one bit of each axis per level, most
+    significant level first."""
+    X = [np.asarray(coords[:, a], dtype=np.int64).copy() for a in range(3)]
+    n = 3
+    top = 1 << (bits - 1)
+    q = top
+    while q > 1:
+        low = q - 1
+        for i in range(n):
+            hit = (X[i] & q) != 0
+            if i == 0:
+                X[0] = np.where(hit, X[0] ^ low, X[0])
+                continue
+            swap = (X[0] ^ X[i]) & low
+            new0 = np.where(hit, X[0] ^ low, X[0] ^ swap)
+            newi = np.where(hit, X[i], X[i] ^ swap)
+            X[0], X[i] = new0, newi
+        q >>= 1
+    for i in range(1, n):
+        X[i] = X[i] ^ X[i - 1]
+    flip = np.zeros_like(X[0])
+    q = top
+    while q > 1:
+        flip = np.where((X[n - 1] & q) != 0, flip ^ (q - 1), flip)
+        q >>= 1
+    for i in range(n):
+        X[i] = X[i] ^ flip
+    idx = np.zeros_like(X[0])
+    for b in range(bits - 1, -1, -1):
+        for i in range(n):
+            idx = (idx << 1) | ((X[i] >> b) & 1)
+    return idx
+
+
+def hilbert_bits(grid):
+    return max(1, int(math.ceil(math.log2(max(grid)))))
+
+
+def hilbert_positions(grid, tile=TILE):
+    """3D Hilbert order: position of each natural token when the valid tokens
+    are sorted by their Hilbert index on the enclosing 2^k cube."""
+    check_grid(grid, tile)
+    key = hilbert_index_3d(token_coords(grid), hilbert_bits(grid))
+    order = np.argsort(key, kind="stable")
+    pos = np.empty_like(order)
+    pos[order] = np.arange(order.size)
+    return pos
+
+
+def positions(grid, order, tile=TILE):
+    if order == "raster":
+        return raster_cube_positions(grid, tile)
+    if order == "hilbert":
+        return hilbert_positions(grid, tile)
+    raise ValueError(order)
+
+
+def tile_cubes(grid, pos, tile=TILE):
+    """Cube coordinate (ct, ch, cw) of every tile rank; raises if a run of 64
+    consecutive positions is not exactly one aligned 4x4x4 cube."""
+    c = token_coords(grid)
+    tsz = tile[0] * tile[1] * tile[2]
+    inv = np.empty_like(pos)
+    inv[pos] = np.arange(pos.size)
+    cube = c[inv] // np.array(tile)
+    cube = cube.reshape(-1, tsz, 3)
+    if not (cube == cube[:, :1, :]).all():
+        raise AssertionError("a tile is not one aligned cube")
+    return cube[:, 0, :]
+
+
+def to_tiled(x, pos):
+    """x[..., N, d] in natural order -> tiled order (row pos[n] <- row n)."""
+    y = np.empty_like(x)
+    y[..., pos, :] = x
+    return y
+
+
+def from_tiled(y, pos):
+    return y[..., pos, :]
+
+
+# ----------------------------------------------------------------------------
+# 3D rotary position encoding
+# ----------------------------------------------------------------------------
+
+def rope_3d(x, coords, dims=(44, 42, 42), base=10000.0):
+    """Rotate x [N, d] (float64) by each token's (t, h, w) coordinate.
+
+    Head dims are split into one group per axis; inside a group of size d_a,
+    pair j = dims (2j, 2j+1) is rotated by angle pos_a * base^(-2j/d_a)."""
+    assert sum(dims) == x.shape[-1]
+    y = np.array(x, dtype=np.float64, copy=True)
+    off = 0
+    for axis, da in enumerate(dims):
+        j = np.arange(da // 2, dtype=np.float64)
+        theta = base ** (-2.0 * j / da)
+        ang = coords[:, axis:axis + 1].astype(np.float64) * theta[None, :]
+        c, s = np.cos(ang), np.sin(ang)
+        x0 = x[:, off + 0:off + da:2].astype(np.float64)
+        x1 = x[:, off + 1:off + da:2].astype(np.float64)
+        y[:, off + 0:off + da:2] = x0 * c - x1 * s
+        y[:, off + 1:off + da:2] = x0 * s + x1 * c
+        off += da
+    return y
+
+
+def round_bf16(x):
+    """Round float64 values to the nearest bf16 value (ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                     # x = m * 2^e, 0.5 <= |m| < 1
+    scaled = np.ldexp(m, 8)                # 8 significant bits
+    r = np.round(scaled)                   # numpy rounds half to even
+    return np.ldexp(r, e - 8)
+
+
+# ----------------------------------------------------------------------------
+# coarse stage: pool, score, softmax, select
+# ----------------------------------------------------------------------------
+
+def pool_tiles(x_tiled, tile_tokens=64):
+    """Mean of each run of 64 tiled rows: [N, d] -> [nT, d]."""
+    N, d = x_tiled.shape
+    return np.asarray(x_tiled, np.float64).reshape(N // tile_tokens, tile_tokens, d).mean(axis=1)
+
+
+def coarse_probabilities(qp, kp, scale):
+    """Row softmax of the pooled logits scale * Qp Kp^T: [nT, nT]."""
+    s = scale * (qp @ kp.T)
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+BORDER = 1e-5
+
+
+def select_blocks(P, top_p, k_min):
+    """Top-p selection with a k_min floor for each row of P [nT, nT].
+
+    Returns counts [nT], idx [nT, nT] (ascending tile ids, -1 padded) and
+    a boolean [nT] marking borderline rows, whose count could change if the
+    cumulative masses moved by 1e-5."""
+    nT = P.shape[1]
+    order = np.argsort(-P, axis=1, kind="stable")       # desc, ties -> lower id
+    cum = np.cumsum(np.take_along_axis(P, order, axis=1), axis=1)
+
+    def count_for(p):
+        if p >= 1.0:
+            return np.full(P.shape[0], nT, np.int64)
+        reach = cum >= p
+        m = np.where(reach.any(axis=1), reach.argmax(axis=1) + 1, nT)
+        return np.minimum(nT, np.maximum(m, max(k_min, 1)))
+
+    counts = count_for(top_p)
+    if top_p >= 1.0:
+        border = np.zeros(P.shape[0], bool)
+    else:
+        border = count_for(top_p + BORDER) != count_for(top_p - BORDER)
+    idx = np.full(P.shape, -1, np.int64)
+    for r in range(P.shape[0]):
+        idx[r, :counts[r]] = np.sort(order[r, :counts[r]])
+    return counts, idx, border
+
+
+def near_tie_rows(P, counts, rel=1e-6):
+    """Rows whose last kept and first dropped probabilities are within rel."""
+    nT = P.shape[1]
+    srt = -np.sort(-P, axis=1)
+    out = np.zeros(P.shape[0], bool)
+    for r in range(P.shape[0]):
+        c = counts[r]
+        if 0 < c < nT:
+            a, b = srt[r, c - 1], srt[r, c]
+            out[r] = abs(a - b) <= rel * max(abs(a), 1e-300)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# fine stage
+# ----------------------------------------------------------------------------
+
+def fine_tile(q_tile, k_tiled, v_tiled, tiles, scale, tile_tokens=64):
+    """Attention of the 64 query rows of one tile over the keys of the given
+    key tiles: out [64, d] and lse [64] (natural log)."""
+    rows = (np.asarray(tiles)[:, None] * tile_tokens + np.arange(tile_tokens)[None, :]).ravel()
+    ks = np.asarray(k_tiled[rows], np.float64)
+    vs = np.asarray(v_tiled[rows], np.float64)
+    s = scale * (np.asarray(q_tile, np.float64) @ ks.T)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ vs) / l, (m + np.log(l))[:, 0]
+
+
+def fine_head(q_tiled, k_tiled, v_tiled, counts, idx, scale, rows=None, tile_tokens=64):
+    """Fine stage of one head in tiled order.  ``rows`` restricts the query
+    tiles computed (others are left NaN)."""
+    N, d = q_tiled.shape
+    out = np.full((N, d), np.nan)
+    lse = np.full(N, np.nan)
+    nT = N // tile_tokens
+    for i in (range(nT) if rows is None else rows):
+        sl = slice(i * tile_tokens, (i + 1) * tile_tokens)
+        out[sl], lse[sl] = fine_tile(q_tiled[sl], k_tiled, v_tiled,
+                                     idx[i, :counts[i]], scale, tile_tokens)
+    return out, lse
+
+
+# ----------------------------------------------------------------------------
+# whole forward pass
+# ----------------------------------------------------------------------------
+
+def as_f64(x, dtype):
+    """Input tensor (bf16 bit patterns as uint16, or float32) -> float64."""
+    if dtype == "bf16":
+        return _bf16_to_f64(x)
+    return np.asarray(x, np.float64)
+
+
+def _bf16_to_f64(x):
+    u = np.asarray(x, np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)
+
+
+def coarse_head(q, k, grid, order, top_p, k_min, scale, rope=None, pos=None):
+    """Steps 1-4 for one head; q, k [N, d] float64 in natural order.
+
+    Returns a dict with the tiled (and, with RoPE, rotated) q/k, pooled
+    Qp/Kp, probabilities, counts, idx and borderline flags."""
+    if pos is None:
+        pos = positions(grid, order)
+    if rope is not None:
+        coords = token_coords(grid)
+        q = rope_3d(q, coords, rope["dims"], rope["base"])
+        k = rope_3d(k, coords, rope["dims"], rope["base"])
+    qt, kt = to_tiled(q, pos), to_tiled(k, pos)
+    qp, kp = pool_tiles(qt), pool_tiles(kt)
+    P = coarse_probabilities(qp, kp, scale)
+    counts, idx, border = select_blocks(P, top_p, k_min)
+    return dict(q_tiled=qt, k_tiled=kt, qp=qp, kp=kp, P=P, counts=counts,
+                idx=idx, border=border, pos=pos)
+
+
+def forward_head(q, k, v, grid, order, top_p, k_min, dtype, scale=None,
+                 rope=None, blocks=None, rows=None):
+    """Whole path for one head, natural order in and out.
+
+    q, k, v: [N, d] as given to the library (bf16 bit patterns or float32).
+    ``blocks`` = (counts, idx) reuses a cached selection (steps 2-4 skipped).
+    ``rows`` restricts the fine stage to the given query tiles."""
+    N, d = q.shape[-2:]
+    if scale is None:
+        scale = default_scale(d)
+    qf, kf, vf = as_f64(q, dtype), as_f64(k, dtype), as_f64(v, dtype)
+    pos = positions(grid, order)
+    res = {}
+    if blocks is None:
+        res = coarse_head(qf, kf, grid, order, top_p, k_min, scale, rope, pos)
+        counts, idx = res["counts"], res["idx"]
+        qt, kt = res["q_tiled"], res["k_tiled"]
+    else:
+        counts, idx = blocks
+        if rope is not None:
+            coords = token_coords(grid)
+            qf = rope_3d(qf, coords, rope["dims"], rope["base"])
+            kf = rope_3d(kf, coords, rope["dims"], rope["base"])
+        qt, kt = to_tiled(qf, pos), to_tiled(kf, pos)
+    if rope is not None and dtype == "bf16":
+        qt, kt = round_bf16(qt), round_bf16(kt)
+    vt = to_tiled(vf, pos)
+    out_t, lse_t = fine_head(qt, kt, vt, counts, idx, scale, rows)
+    res.update(out=from_tiled(out_t, pos), lse=lse_t[pos], out_tiled=out_t,
+               lse_tiled=lse_t, counts=counts, idx=idx, pos=pos)
+    return res
+
+
+def dense_attention_loop(q, k, v, scale):
+    """Independent O(N^2) dense softmax attention with plain Python loops
+    (tiny inputs only): out [N, d], lse [N]."""
+    N, d = len(q), len(q[0])
+    out, lse = [], []
+    for i in range(N):
+        logits = [scale * sum(q[i][c] * k[j][c] for c in range(d)) for j in range(N)]
+        m = max(logits)
+        w = [math.exp(x - m) for x in logits]
+        z = math.fsum(w)
+        out.append([math.fsum(w[j] * v[j][c] for j in range(N)) / z for c in range(d)])
+        lse.append(m + math.log(z))
+    return out, lse
