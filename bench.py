@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of adaptive block-sparse spatiotemporal attention on B200.
+
+Metric: sparse-attention forward ms and effective TFLOP/s at the Wan-480p
+latent (20x32x52 = 33,280 tokens, 40 heads, d=128, bf16, top-p 0.95,
+k_min 8).  One step = one ``fvattn_forward`` call: pool/select, schedule and
+the block-sparse fine stage over one batch of synthetic input (the tile
+reorder and its inverse are fused into the loads and stores).  Effective
+FLOPs = 4 * 64 * 64 * d per selected (query tile, key tile) pair.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fvattn|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent
+replica of the workload (heads shard with no exchange), the time is the max
+over ranks and ``value`` counts the work of all ranks ("scaling": "weak").
+``--impl reference`` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_spatiotemporal_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "sparse-attn fwd ms & effective TFLOP/s (33k tok, 40 heads, d=128, top-p .95)"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def pair_flops(d: int) -> float:
+    return 4.0 * 64 * 64 * d
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ("block_sparse_spatiotemporal_b200/csrc/fine_tc.cu",
+                "block_sparse_spatiotemporal_b200/csrc/fvattn_internal.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """dram bytes per fine-kernel launch from the committed ncu summary, or
+    None when the summary is absent or was taken on another kernel source."""
+    path = os.path.join(ROOT, "profiles", f"fine_tc_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpus):
+        self.gpus = set(gpus)
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or not f[0].isdigit() or int(f[0]) not in self.gpus:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, q, k, v, budget_s: float, seed: int = 0):
+    """Time the oracle as it stands on a bounded sample: the coarse stage of
+    every head, then the fine stage of randomly drawn (head, query tile)
+    rows until the budget is spent.  Returns (est_full_seconds, flops_full,
+    description, threads)."""
+    from oracle import fvattn_oracle as O
+    rope = dict(dims=wl.rope_dims, base=wl.rope_base) if wl.rope else None
+    pos = O.positions(wl.grid, wl.order)
+    scale = O.default_scale(wl.head_dim)
+    t0 = time.perf_counter()
+    coarse = []
+    coarse_heads = 0
+    for h in range(wl.heads):
+        coarse.append(O.coarse_head(O.as_f64(q[0, h], wl.dtype), O.as_f64(k[0, h], wl.dtype), wl.grid, wl.order,
+                                    wl.top_p, wl.k_min, scale, rope, pos))
+        coarse_heads += 1
+        if time.perf_counter() - t0 > budget_s / 2 and h < wl.heads - 1:
+            break
+    t_coarse = time.perf_counter() - t0
+    pairs_per_head = [int(r["counts"].sum()) for r in coarse]
+    est_pairs_total = sum(pairs_per_head) * wl.heads / coarse_heads
+    rng = np.random.default_rng(seed)
+    t1 = time.perf_counter()
+    done_pairs = 0
+    rows = 0
+    vt_cache = {}
+    while time.perf_counter() - t1 < budget_s / 2 or rows == 0:
+        h = int(rng.integers(coarse_heads))
+        i = int(rng.integers(wl.num_tiles))
+        r = coarse[h]
+        if h not in vt_cache:
+            qt, kt = r["q_tiled"], r["k_tiled"]
+            if wl.rope and wl.dtype == "bf16":
+                qt, kt = O.round_bf16(qt), O.round_bf16(kt)
+            vt_cache = {h: (qt, kt, O.to_tiled(O.as_f64(v[0, h], wl.dtype), pos))}
+        qt, kt, vt = vt_cache[h]
+        O.fine_tile(qt[i * 64:(i + 1) * 64], kt, vt, r["idx"][i, :r["counts"][i]], scale)
+        done_pairs += int(r["counts"][i])
+        rows += 1
+    t_fine = time.perf_counter() - t1
+    est = t_coarse * wl.heads / coarse_heads + t_fine * est_pairs_total / max(done_pairs, 1)
+    desc = (f"oracle (numpy fp64) coarse stage of {coarse_heads}/{wl.heads} heads + fine stage of {rows} random "
+            f"(head, query tile) rows ({done_pairs} selected pairs of ~{int(est_pairs_total)}), scaled to the full "
+            f"workload by heads and by selected pairs")
+    flops = est_pairs_total * pair_flops(wl.head_dim)
+    return est, flops, desc, _threads()
+
+
+def _threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((x.get("num_threads", 1) for x in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v = make_inputs(wl)
+    per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wl, q, k, v, min(per_step, 2.0), seed=1)
+    secs, flops = [], None
+    desc, cores = "", 1
+    for s in range(args.steps):
+        est, flops, desc, cores = oracle_sample(wl, q, k, v, per_step, seed=100 + s)
+        secs.append(est)
+    ms = 1000.0 * statistics.mean(secs)
+    value = flops / (ms / 1000.0) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "grid": list(wl.grid), "heads": wl.heads, "head_dim": wl.head_dim,
+                       "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, wl):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    q, k, v = make_inputs(wl)
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
+    shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16,
+                         order=F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE)
+    rope = F.make_rope(wl.rope_dims, wl.rope_base) if wl.rope else None
+    ws = F.workspace(shape, rope, device=dev)
+    cache, counts, _ = F.new_cache(shape, device=dev)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qx=qd, kx=kd, vx=vd):
+        F.forward(shape, qx, kx, vx, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=out, lse=lse)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize(dev)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+    pairs = int(counts.sum().item())
+    flops_step = pairs * pair_flops(wl.head_dim)
+
+    # ---- timed region (device time, CUDA events on the launch stream)
+    sampler = ClockSampler(range(world)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    F.profile_read()
+    F.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    F.profile_enable(False)
+    stages = F.profile_read()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during the timed region")
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end through the public API: pinned host in, host out
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        qb, kb, vb = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+        for _ in range(2):
+            qb.copy_(qh, non_blocking=True); kb.copy_(kh, non_blocking=True); vb.copy_(vh, non_blocking=True)
+            step(qb, kb, vb)
+            oh.copy_(out, non_blocking=True)
+        n_e2e = max(3, min(args.steps, 20))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_e2e):
+            qb.copy_(qh, non_blocking=True); kb.copy_(kh, non_blocking=True); vb.copy_(vh, non_blocking=True)
+            step(qb, kb, vb)
+            oh.copy_(out, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        t2 = torch.tensor([s0.elapsed_time(s1) / n_e2e], device=dev)
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t2.item())
+        h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+        d2h = oh.numel() * oh.element_size()
+        e2e = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        fine_ms, fine_n = stages["fine"]
+        fine_avg = fine_ms / max(fine_n, 1)
+        achieved = flops_step / (fine_avg / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        traffic = profiled_traffic(wl.name)
+        stage_ms = {name: round(v[0] / max(args.steps, 1), 4) for name, v in stages.items() if v[1]}
+        pool_select_ms = (stages["pool"][0] + stages["select"][0]) / args.steps
+        qk_bytes = 2 * wl.heads * wl.tokens * wl.head_dim * 2
+        line = {
+            "metric": METRIC,
+            "value": world * flops_step / (ms_max / 1e3) / 1e12,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "grid": list(wl.grid), "tokens": wl.tokens, "heads": wl.heads,
+                       "head_dim": wl.head_dim, "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order,
+                       "rope": wl.rope, "selected_pairs": pairs,
+                       "density": pairs / (wl.heads * wl.num_tiles ** 2),
+                       "l2": "inputs larger than L2 (q+k+v = %.0f MB)" % (3 * qk_bytes / 2 / 1e6),
+                       "parallelism": f"replica x{world}"},
+            "stage_ms": stage_ms,
+            "pool_select": {"ms": pool_select_ms, "gbs": qk_bytes / (pool_select_ms / 1e3) / 1e9,
+                            "frac_of_hbm": qk_bytes / (pool_select_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+            "roofline": {"kernel": "fine_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{pk_kind} bf16 burst"},
+            "gpu_launches": sum(n for _, n in stages.values()) + args.steps * (1 if rope is None else 2),
+            "clocks": clocks,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            est, flops, desc, cores = oracle_sample(wl, q, k, v, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": flops / est / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": desc, "est_ms_per_step": est * 1e3}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("fvattn", "reference"), default="fvattn")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="wan480p")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

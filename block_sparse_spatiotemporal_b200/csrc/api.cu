@@ -1,0 +1,536 @@
+// C-ABI entry points of libfvattn.so (declared in include/fvattn.h): host-side
+// validation, workspace carve-up, TMA descriptors and the launch sequence of
+// each call.  No entry point allocates device memory.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "fvattn_internal.cuh"
+
+using namespace fvattn;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+int map_cuda(cudaError_t e) { return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA; }
+
+#define FV_TRY(expr)                          \
+  do {                                        \
+    const int _st = (expr);                   \
+    if (_st != FVATTN_OK) return _st;         \
+  } while (0)
+#define FV_CUDA(expr) FV_TRY(map_cuda(expr))
+
+int elem_size(int dtype) { return dtype == FVATTN_BF16 ? 2 : 4; }
+
+int make_geom(const fvattn_shape* s, Geom* g) {
+  if (!s) return FVATTN_ERR_INVALID_ARG;
+  if (s->dtype != FVATTN_F32 && s->dtype != FVATTN_BF16) return FVATTN_ERR_DTYPE;
+  if (s->order != FVATTN_ORDER_RASTER_CUBE && s->order != FVATTN_ORDER_HILBERT) return FVATTN_ERR_INVALID_ARG;
+  if (s->layout != FVATTN_LAYOUT_NATURAL && s->layout != FVATTN_LAYOUT_TILED) return FVATTN_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->heads < 1) return FVATTN_ERR_SHAPE;
+  if (s->tile.t != 4 || s->tile.h != 4 || s->tile.w != 4) return FVATTN_ERR_SHAPE;
+  const int T = s->grid.T, Hg = s->grid.H, W = s->grid.W;
+  if (T < 4 || Hg < 4 || W < 4 || T % 4 || Hg % 4 || W % 4 || T > 4096 || Hg > 4096 || W > 4096)
+    return FVATTN_ERR_SHAPE;
+  const int d = s->head_dim;
+  if (s->dtype == FVATTN_BF16) {
+    if (d == 32 || d == 64) return FVATTN_ERR_UNSUPPORTED;
+    if (d != 128) return FVATTN_ERR_SHAPE;
+  } else if (d != 32 && d != 64 && d != 128) {
+    return FVATTN_ERR_SHAPE;
+  }
+  const long long N = (long long)T * Hg * W;
+  const long long nT = N / 64;
+  if (nT > 4096) return FVATTN_ERR_SHAPE;
+  const long long BH = (long long)s->batch * s->heads;
+  if (BH * N * d >= (1ll << 31)) return FVATTN_ERR_SHAPE;
+  if (std::isnan(s->scale) || s->scale < 0.f || std::isinf(s->scale)) return FVATTN_ERR_INVALID_ARG;
+  g->B = s->batch;
+  g->H = s->heads;
+  g->d = d;
+  g->T = T;
+  g->Hg = Hg;
+  g->W = W;
+  g->nt = T / 4;
+  g->nh = Hg / 4;
+  g->nw = W / 4;
+  g->nT = (int)nT;
+  g->N = (int)N;
+  g->BH = (int)BH;
+  g->P = (int)((nT + 1) / 2);
+  g->order = s->order;
+  g->scale = s->scale > 0.f ? s->scale : (float)(1.0 / std::sqrt((double)d));
+  return FVATTN_OK;
+}
+
+bool rope_on(const fvattn_rope* r) { return r && r->enabled; }
+
+int check_rope(const fvattn_rope* r, const Geom& g) {
+  if (!rope_on(r)) return FVATTN_OK;
+  if (r->dt < 0 || r->dh < 0 || r->dw < 0 || (r->dt | r->dh | r->dw) & 1) return FVATTN_ERR_INVALID_ARG;
+  if (r->dt + r->dh + r->dw != g.d) return FVATTN_ERR_INVALID_ARG;
+  if (!(r->base > 0.f) || std::isinf(r->base)) return FVATTN_ERR_INVALID_ARG;
+  return FVATTN_OK;
+}
+
+WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.tile_cube = take(sizeof(int) * g.nT);
+  L.cube_rank = take(sizeof(int) * g.nT);
+  L.tile_tok = take(sizeof(int) * (size_t)g.N);
+  const size_t rope_pairs =
+      rope_on(r) ? (size_t)g.T * (r->dt / 2) + (size_t)g.Hg * (r->dh / 2) + (size_t)g.W * (r->dw / 2) : 0;
+  L.rope_tab = take(sizeof(float2) * rope_pairs);
+  L.qp = take(sizeof(float) * (size_t)g.BH * g.nT * g.d);
+  L.kp = take(sizeof(float) * (size_t)g.BH * g.nT * g.d);
+  L.counts = take(sizeof(int) * (size_t)g.BH * g.nT);
+  L.idx = take(sizeof(int) * (size_t)g.BH * g.nT * g.nT);
+  L.uni = take(sizeof(int) * (size_t)g.BH * g.P * g.nT);
+  L.ucount = take(sizeof(int) * (size_t)g.BH * g.P);
+  L.worklist = take(sizeof(int) * (size_t)g.BH * g.P);
+  const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
+  L.qrot = take(rot);
+  L.krot = take(rot);
+  L.total = off;
+  return L;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+};
+
+int device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = 0;
+  FV_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return FVATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev].sms == 0) {
+    FV_CUDA(cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev));
+    FV_CUDA(cudaDeviceGetAttribute(&cache[dev].major, cudaDevAttrComputeCapabilityMajor, dev));
+  }
+  *out = cache[dev];
+  if (out->major != 10) return FVATTN_ERR_UNSUPPORTED;
+  return FVATTN_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// TMA descriptor over a bf16 [BH, N, 128] tensor, box = one 64-token tile x
+// 64 head dims, 128-byte swizzle.  natural: 5D (d, W, Hg, T, BH) with a
+// 64 x 4 x 4 x 4 box (one aligned cube); tiled: 3D (d, N, BH), 64 x 64 box.
+int make_tile_map(CUtensorMap* map, const void* base, const Geom& g, bool natural) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FVATTN_ERR_CUDA;
+  const cuuint64_t row = (cuuint64_t)g.d * 2;
+  CUresult r;
+  if (natural) {
+    const cuuint64_t dims[5] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.Hg, (cuuint64_t)g.T,
+                                (cuuint64_t)g.BH};
+    const cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.Hg, row * (cuuint64_t)g.N};
+    const cuuint32_t box[5] = {64, 4, 4, 4, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+    const cuuint64_t strides[2] = {row, row * (cuuint64_t)g.N};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Optional per-stage timing with CUDA events (host objects only).
+// ---------------------------------------------------------------------------
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec { int stage; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+
+// Records events around one launch when profiling is on.
+struct StageTimer {
+  int stage;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  StageTimer(int st, cudaStream_t stream) : stage(st), s(stream) {
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (!p.on) return;
+    a = p.get();
+    b = p.get();
+    if (a && b) cudaEventRecord(a, s);
+  }
+  ~StageTimer() {
+    if (!a || !b) return;
+    cudaEventRecord(b, s);
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> lock(p.mu);
+    p.recs.push_back({stage, a, b});
+  }
+};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Common prologue: shape, workspace, device.
+struct Call {
+  Geom g{};
+  WsLayout L{};
+  DeviceInfo dev{};
+  char* ws = nullptr;
+  int* status = nullptr;
+  cudaStream_t s = nullptr;
+
+  template <typename T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+};
+
+int begin(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws, size_t ws_bytes,
+          fvattn_stream_t stream) {
+  FV_TRY(make_geom(shape, &c->g));
+  FV_TRY(check_rope(rope, c->g));
+  if (!ws || !aligned(ws, kAlign)) return FVATTN_ERR_INVALID_ARG;
+  c->L = layout_for(c->g, shape->dtype, rope);
+  if (ws_bytes < c->L.total) return FVATTN_ERR_WORKSPACE;
+  FV_TRY(device_info(&c->dev));
+  c->ws = static_cast<char*>(ws);
+  c->status = c->at<int>(c->L.status);
+  c->s = reinterpret_cast<cudaStream_t>(stream);
+  FV_CUDA(cudaMemsetAsync(c->status, 0, sizeof(int), c->s));
+  return FVATTN_OK;
+}
+
+int tables(const Call& c, const fvattn_rope* rope, bool need_tok) {
+  StageTimer t(FVATTN_STAGE_TABLES, c.s);
+  FV_CUDA(launch_tile_table(c.g, c.at<int>(c.L.tile_cube), c.at<int>(c.L.cube_rank), c.s));
+  if (need_tok) FV_CUDA(launch_tile_token(c.g, c.at<int>(c.L.cube_rank), c.at<int>(c.L.tile_tok), c.s));
+  if (rope_on(rope))
+    FV_CUDA(launch_rope_table(c.g, rope->dt, rope->dh, rope->dw, rope->base, c.at<float2>(c.L.rope_tab), c.s));
+  return FVATTN_OK;
+}
+
+int check_blocks(const fvattn_blocks* b, const Geom& g) {
+  if (!b || !b->counts || !b->idx) return FVATTN_ERR_INVALID_ARG;
+  if (!aligned(b->counts, 4) || !aligned(b->idx, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (b->cap < g.nT) return FVATTN_ERR_CAPACITY;
+  return FVATTN_OK;
+}
+
+// Pool (+ RoPE) and select into `blocks`; writes rotated copies if asked.
+int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
+               bool natural, bool pooled, bool rot, float top_p, int k_min, const fvattn_blocks* blocks) {
+  const bool r = rope_on(rope);
+  {
+  StageTimer t(FVATTN_STAGE_POOL, c.s);
+  FV_CUDA(launch_pool(c.g, shape->dtype, q, k, natural ? 1 : 0, c.at<int>(c.L.tile_cube), c.at<int>(c.L.tile_tok),
+                      r ? 1 : 0, r ? rope->dt : 0, r ? rope->dh : 0, r ? rope->dw : 0, c.at<float2>(c.L.rope_tab),
+                      pooled ? c.at<float>(c.L.qp) : nullptr, pooled ? c.at<float>(c.L.kp) : nullptr,
+                      rot ? c.at<void>(c.L.qrot) : nullptr, rot ? c.at<void>(c.L.krot) : nullptr, c.s));
+  }
+  StageTimer t(FVATTN_STAGE_SELECT, c.s);
+  if (pooled)
+    FV_CUDA(launch_select(c.g, c.at<float>(c.L.qp), c.at<float>(c.L.kp), top_p, k_min, blocks->counts, blocks->idx,
+                          blocks->cap, c.s));
+  return FVATTN_OK;
+}
+
+int run_schedule(const Call& c, const fvattn_blocks* blocks, int* worklist) {
+  StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
+  FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
+                       c.status, c.s));
+  FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, worklist, c.s));
+  return FVATTN_OK;
+}
+
+// Fine stage.  q/k come from the rotated tiled copies when RoPE is on.
+int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const void* v,
+             const fvattn_rope* rope, bool natural, const fvattn_blocks* blocks, void* out, float* lse) {
+  const bool r = rope_on(rope);
+  const void* qs = r ? c.at<void>(c.L.qrot) : q;
+  const void* ks = r ? c.at<void>(c.L.krot) : k;
+  const bool qk_nat = natural && !r;
+  if (shape->dtype == FVATTN_BF16) {
+    CUtensorMap mq, mk, mv;
+    FV_TRY(make_tile_map(&mq, qs, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mk, ks, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mv, v, c.g, natural));
+    FineTcArgs a{};
+    a.g = c.g;
+    a.uni = c.at<int>(c.L.uni);
+    a.ucount = c.at<int>(c.L.ucount);
+    a.worklist = c.at<int>(c.L.worklist);
+    a.n_items = c.g.BH * c.g.P;
+    a.tile_cube = c.at<int>(c.L.tile_cube);
+    a.q_nat = qk_nat;
+    a.k_nat = qk_nat;
+    a.v_nat = natural;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.out_nat = natural;
+    a.status = c.status;
+    a.wait_cap = kDefaultWaitCap;
+    StageTimer t(FVATTN_STAGE_FINE, c.s);
+    FV_CUDA(launch_fine_tc(mq, mk, mv, a, c.dev.sms, c.s));
+  } else {
+    FineF32Args a{};
+    a.g = c.g;
+    a.q = static_cast<const float*>(qs);
+    a.k = static_cast<const float*>(ks);
+    a.v = static_cast<const float*>(v);
+    a.q_nat = qk_nat;
+    a.k_nat = qk_nat;
+    a.v_nat = natural;
+    a.counts = blocks->counts;
+    a.idx = blocks->idx;
+    a.cap = blocks->cap;
+    a.tile_cube = c.at<int>(c.L.tile_cube);
+    a.out = static_cast<float*>(out);
+    a.lse = lse;
+    a.out_nat = natural;
+    a.status = c.status;
+    StageTimer t(FVATTN_STAGE_FINE, c.s);
+    FV_CUDA(launch_fine_f32(a, c.s));
+  }
+  return FVATTN_OK;
+}
+
+bool same_shape(const fvattn_shape& a, const fvattn_shape& b) {
+  return a.batch == b.batch && a.heads == b.heads && a.head_dim == b.head_dim && a.grid.T == b.grid.T &&
+         a.grid.H == b.grid.H && a.grid.W == b.grid.W && a.tile.t == b.tile.t && a.tile.h == b.tile.h &&
+         a.tile.w == b.tile.w && a.dtype == b.dtype && a.order == b.order;
+}
+
+bool tensor_ok(const void* p) { return p && aligned(p, 16); }
+
+}  // namespace
+
+extern "C" {
+
+int fvattn_num_tiles(const fvattn_shape* shape, int64_t* num_tiles) {
+  Geom g;
+  if (!num_tiles) return FVATTN_ERR_INVALID_ARG;
+  FV_TRY(make_geom(shape, &g));
+  *num_tiles = g.nT;
+  return FVATTN_OK;
+}
+
+int fvattn_workspace_size(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes) {
+  Geom g;
+  if (!bytes) return FVATTN_ERR_INVALID_ARG;
+  FV_TRY(make_geom(shape, &g));
+  FV_TRY(check_rope(rope, g));
+  *bytes = layout_for(g, shape->dtype, rope).total;
+  return FVATTN_OK;
+}
+
+int fvattn_tile_reorder(const fvattn_shape* shape, const void* x, void* y, int32_t row_bytes, int inverse, void* ws,
+                        size_t ws_bytes, fvattn_stream_t stream) {
+  if (!tensor_ok(x) || !tensor_ok(y) || x == y) return FVATTN_ERR_INVALID_ARG;
+  if (row_bytes < 4 || row_bytes > 1024 || row_bytes % 4) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, nullptr, ws, ws_bytes, stream));
+  FV_TRY(tables(c, nullptr, false));
+  StageTimer t(FVATTN_STAGE_REORDER, c.s);
+  FV_CUDA(launch_reorder(c.g, c.at<int>(c.L.cube_rank), x, y, row_bytes, inverse ? 1 : 0, c.dev.sms, c.s));
+  return FVATTN_OK;
+}
+
+int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope, float top_p,
+                       int32_t k_min, const fvattn_blocks* out, void* ws, size_t ws_bytes, fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k)) return FVATTN_ERR_INVALID_ARG;
+  if (std::isnan(top_p) || k_min < 0) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream));
+  FV_TRY(check_blocks(out, c.g));
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
+  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, false, top_p, k_min, out));
+  return FVATTN_OK;
+}
+
+int fvattn_build_worklist(const fvattn_shape* shape, const fvattn_blocks* blocks, int32_t* worklist, void* ws,
+                          size_t ws_bytes, fvattn_stream_t stream) {
+  if (!worklist || !aligned(worklist, 4)) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, nullptr, ws, ws_bytes, stream));
+  FV_TRY(check_blocks(blocks, c.g));
+  FV_TRY(run_schedule(c, blocks, worklist));
+  return FVATTN_OK;
+}
+
+int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void* k, const void* v,
+                            const fvattn_rope* rope, const fvattn_blocks* blocks, void* out, float* lse, void* ws,
+                            size_t ws_bytes, fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(out) || !lse || !aligned(lse, 4))
+    return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream));
+  FV_TRY(check_blocks(blocks, c.g));
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
+  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
+  FV_TRY(run_schedule(c, blocks, c.at<int>(c.L.worklist)));
+  FV_TRY(run_fine(c, shape, q, k, v, rope, natural, blocks, out, lse));
+  return FVATTN_OK;
+}
+
+int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, const void* v, const fvattn_rope* rope,
+                   float top_p, int32_t k_min, fvattn_mask_cache* cache, int reuse_mask, void* out, float* lse,
+                   void* ws, size_t ws_bytes, fvattn_stream_t stream) {
+  if (!shape) return FVATTN_ERR_INVALID_ARG;
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(out) || !lse || !aligned(lse, 4))
+    return FVATTN_ERR_INVALID_ARG;
+  if (std::isnan(top_p) || k_min < 0) return FVATTN_ERR_INVALID_ARG;
+  fvattn_shape sh = *shape;
+  sh.layout = FVATTN_LAYOUT_NATURAL;
+  Call c;
+  FV_TRY(begin(&c, &sh, rope, ws, ws_bytes, stream));
+  fvattn_blocks local{c.at<int>(c.L.counts), c.at<int>(c.L.idx), c.g.nT};
+  const fvattn_blocks* blocks = &local;
+  if (reuse_mask) {
+    if (!cache || !cache->valid || !same_shape(cache->shape, sh)) return FVATTN_ERR_CACHE_MISMATCH;
+    blocks = &cache->blocks;
+    FV_TRY(check_blocks(blocks, c.g));
+  } else if (cache) {
+    blocks = &cache->blocks;
+    FV_TRY(check_blocks(blocks, c.g));
+  }
+  FV_TRY(tables(c, rope, false));
+  if (!reuse_mask) {
+    FV_TRY(run_coarse(c, &sh, q, k, rope, true, true, rope_on(rope), top_p, k_min, blocks));
+  } else if (rope_on(rope)) {
+    FV_TRY(run_coarse(c, &sh, q, k, rope, true, false, true, 0.f, 0, blocks));
+  }
+  FV_TRY(run_schedule(c, blocks, c.at<int>(c.L.worklist)));
+  FV_TRY(run_fine(c, &sh, q, k, v, rope, true, blocks, out, lse));
+  if (cache && !reuse_mask) {
+    cache->shape = sh;
+    cache->top_p = top_p;
+    cache->k_min = k_min;
+    cache->valid = 1;
+  }
+  return FVATTN_OK;
+}
+
+int fvattn_get_device_status(void* ws, fvattn_stream_t stream, int32_t* status) {
+  if (!ws || !status) return FVATTN_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FV_CUDA(cudaStreamSynchronize(s));
+  int v = 0;
+  FV_CUDA(cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost));
+  FV_CUDA(cudaMemset(ws, 0, sizeof(int)));
+  *status = v;
+  return FVATTN_OK;
+}
+
+int fvattn_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t cap_iterations, fvattn_stream_t stream) {
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < kAlign || cap_iterations < 1) return FVATTN_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  FV_TRY(device_info(&dev));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FV_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  FV_CUDA(launch_wait_selftest(static_cast<int*>(ws), cap_iterations, s));
+  return FVATTN_OK;
+}
+
+int fvattn_profile_enable(int enable) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lock(p.mu);
+  p.on = enable != 0;
+  return FVATTN_OK;
+}
+
+int fvattn_profile_read(double* ms, int64_t* launches) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lock(p.mu);
+  double acc[FVATTN_STAGE_COUNT] = {0};
+  int64_t cnt[FVATTN_STAGE_COUNT] = {0};
+  int st = FVATTN_OK;
+  for (auto& r : p.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = FVATTN_ERR_CUDA;
+    acc[r.stage] += t;
+    cnt[r.stage] += 1;
+    p.pool.push_back(r.a);
+    p.pool.push_back(r.b);
+  }
+  p.recs.clear();
+  for (int i = 0; i < FVATTN_STAGE_COUNT; ++i) {
+    if (ms) ms[i] = acc[i];
+    if (launches) launches[i] = cnt[i];
+  }
+  return st;
+}
+
+const char* fvattn_status_string(int status) {
+  switch (status) {
+    case FVATTN_OK: return "ok";
+    case FVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FVATTN_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case FVATTN_ERR_DTYPE: return "unsupported dtype";
+    case FVATTN_ERR_CAPACITY: return "block list capacity smaller than the number of tiles";
+    case FVATTN_ERR_CUDA: return "CUDA call failed";
+    case FVATTN_ERR_CACHE_MISMATCH: return "mask cache not valid for this shape";
+    case FVATTN_ERR_DEVICE: return "a kernel reported an error";
+    case FVATTN_ERR_WORKSPACE: return "workspace too small";
+    case FVATTN_ERR_UNSUPPORTED: return "unsupported device or combination";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,294 @@
+// Internal declarations shared by the fvattn CUDA sources (sm_100a only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fvattn.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "fvattn kernels are written for sm_100a (B200) only"
+#endif
+
+namespace fvattn {
+
+constexpr int kTileTokens = 64;
+constexpr int kMaxTiles = 8192;
+
+// Device status codes (workspace status word).
+constexpr int kStatusBadBlock = 1;
+constexpr int kStatusWaitCap = 2;
+
+// Default iteration cap of a bounded wait: on the order of a second.
+constexpr long long kDefaultWaitCap = 1ll << 24;
+
+// ---------------------------------------------------------------------------
+// Problem geometry passed to kernels by value.
+// ---------------------------------------------------------------------------
+struct Geom {
+  int B, H, d;
+  int T, Hg, W;          // latent grid
+  int nt, nh, nw;        // tile grid
+  int nT;                // tiles per head
+  int N;                 // tokens per head
+  int BH;
+  int P;                 // query-tile pairs per head = ceil(nT/2)
+  int order;             // fvattn_order
+  float scale;           // softmax scale
+};
+
+// Workspace carve-up (byte offsets from the workspace base).
+struct WsLayout {
+  size_t status;         // int32 status word + padding
+  size_t tile_cube;      // int32 [nT]: packed (ct<<20 | ch<<10 | cw) of tile rank j
+  size_t cube_rank;      // int32 [nT]: tile rank of raster cube id
+  size_t tile_tok;       // int32 [N]: natural token index of each tiled row
+  size_t rope_tab;       // float2 [(T*dt + Hg*dh + W*dw)/2]: (cos, sin)
+  size_t qp, kp;         // float [BH*nT*d]
+  size_t counts, idx;    // int32 [BH*nT], [BH*nT*nT] (forward without cache)
+  size_t uni, ucount;    // int32 [BH*P*nT], [BH*P]
+  size_t worklist;       // int32 [BH*P]
+  size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
+  size_t total;
+};
+
+// Kernel arguments filled by the host entry points.
+struct RopeArgs {
+  int enabled, dt, dh, dw;
+  const float2* tab;     // [T*dt/2 | Hg*dh/2 | W*dw/2]
+};
+
+struct FineTcArgs {
+  Geom g;
+  const int* uni;
+  const int* ucount;
+  const int* worklist;
+  int n_items;
+  const int* tile_cube;
+  int q_nat, k_nat, v_nat;
+  __nv_bfloat16* out;
+  float* lse;
+  int out_nat;
+  int* status;
+  long long wait_cap;
+};
+
+struct FineF32Args {
+  Geom g;
+  const float* q;
+  const float* k;
+  const float* v;
+  int q_nat, k_nat, v_nat;
+  const int* counts;
+  const int* idx;
+  int cap;
+  const int* tile_cube;
+  float* out;
+  float* lse;
+  int out_nat;
+  int* status;
+};
+
+__host__ __device__ inline int pack_cube(int ct, int ch, int cw) { return (ct << 20) | (ch << 10) | cw; }
+__host__ __device__ inline int cube_t(int p) { return p >> 20; }
+__host__ __device__ inline int cube_h(int p) { return (p >> 10) & 1023; }
+__host__ __device__ inline int cube_w(int p) { return p & 1023; }
+
+// Natural token index of row r (0..63, raster inside the cube) of a cube.
+__device__ inline int cube_row_token(const Geom& g, int packed, int r) {
+  int t = cube_t(packed) * 4 + (r >> 4);
+  int h = cube_h(packed) * 4 + ((r >> 2) & 3);
+  int w = cube_w(packed) * 4 + (r & 3);
+  return (t * g.Hg + h) * g.W + w;
+}
+
+__device__ inline void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers: shared-memory addresses, mbarriers, TMA, tcgen05.
+// ---------------------------------------------------------------------------
+__device__ inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ inline void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Gives up after `cap`
+// polls, or as soon as another thread of the block raised `abort`; on
+// giving up it raises `abort`, records kStatusWaitCap and returns false.
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                 long long cap) {
+  for (long long i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 255 && *abort) return false;
+    if (i >= cap) {
+      *abort = 1;
+      set_status(status, kStatusWaitCap);
+      return false;
+    }
+  }
+}
+
+__device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                   int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ inline void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                   int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
+__device__ inline void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// tcgen05 --------------------------------------------------------------------
+__device__ inline void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ inline void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ inline void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]
+__device__ inline void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ inline void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ inline void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ inline void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ inline void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// UMMA shared-memory matrix descriptor, 128-byte swizzle, sm_100 version 1.
+//   start: byte address in shared memory; lbo/sbo: byte offsets.
+__device__ inline uint64_t umma_desc_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;            // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                       // D format: f32
+         | (1u << 7)                     // A format: bf16
+         | (1u << 10)                    // B format: bf16
+         | ((a_mn_major ? 1u : 0u) << 15)
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (one per kernel family); each returns the launch error.
+// ---------------------------------------------------------------------------
+cudaError_t launch_tile_table(const Geom& g, int* tile_cube, int* cube_rank, cudaStream_t s);
+cudaError_t launch_tile_token(const Geom& g, const int* cube_rank, int* tile_tok, cudaStream_t s);
+cudaError_t launch_reorder(const Geom& g, const int* cube_rank, const void* x, void* y, int row_bytes, int inverse,
+                           int num_sms, cudaStream_t s);
+cudaError_t launch_rope_table(const Geom& g, int dt, int dh, int dw, float base, float2* tab, cudaStream_t s);
+cudaError_t launch_pool(const Geom& g, int dtype, const void* q, const void* k, int natural, const int* tile_cube,
+                        const int* tile_tok, int rope_enabled, int dt, int dh, int dw, const float2* rope_tab,
+                        float* qp, float* kp, void* qrot, void* krot, cudaStream_t s);
+cudaError_t launch_select(const Geom& g, const float* qp, const float* kp, float top_p, int k_min, int* counts,
+                          int* idx, int cap, cudaStream_t s);
+cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
+                         cudaStream_t s);
+cudaError_t launch_rank(const int* key, int n, int* worklist, cudaStream_t s);
+cudaError_t launch_fine_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineTcArgs& a,
+                           int num_sms, cudaStream_t s);
+cudaError_t launch_fine_f32(const FineF32Args& a, cudaStream_t s);
+cudaError_t launch_wait_selftest(int* status, long long cap, cudaStream_t s);
+
+}  // namespace fvattn

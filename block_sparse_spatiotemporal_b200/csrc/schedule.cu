@@ -1,0 +1,108 @@
+// Fine-stage schedule: the single-GPU analogue of the "FVAttn" digest's
+// runtime head-level load balancing (section 02), applied across the SMs of
+// one GPU instead of across GPUs.
+//
+// A work item is a pair of adjacent query tiles (2p, 2p+1) of one (batch,
+// head): the pair fills the 128 rows of one tensor-core tile, and the item
+// walks the union of the two tiles' key lists, each entry tagged with which
+// tile selected it (the other tile's rows are masked for that key tile).
+// Items are then ranked by union size, longest first (LPT), ties by item
+// code, so the persistent fine kernel hands the heavy items out first and
+// the light ones fill the tail.
+#include "fvattn_internal.cuh"
+
+namespace fvattn {
+
+// One warp per item.  Entries: tile | (mask << 16), mask bit 0 = tile 2p
+// selected it, bit 1 = tile 2p+1.  Ascending tile ids.  Validates the lists:
+// counts in [0, nT], ids in [0, nT) and strictly ascending; violations set
+// kStatusBadBlock and the offending entries are dropped.
+__global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restrict__ counts,
+                                                    const int* __restrict__ idx, int cap, int* __restrict__ uni,
+                                                    int* __restrict__ ucount, int* status) {
+  extern __shared__ uint32_t bm[];  // per warp: 2 bitmaps of ceil(nT/32) words
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int words = (g.nT + 31) / 32;
+  uint32_t* bma = bm + warp * 2 * words;
+  uint32_t* bmb = bma + words;
+  const long long item = (long long)blockIdx.x * 4 + warp;
+  if (item >= (long long)g.BH * g.P) return;
+  const int bh = (int)(item / g.P), p = (int)(item % g.P);
+  for (int w = lane; w < 2 * words; w += 32) bma[w] = 0u;
+  __syncwarp();
+  for (int half = 0; half < 2; ++half) {
+    const int tile = 2 * p + half;
+    if (tile >= g.nT) break;
+    const size_t row = (size_t)bh * g.nT + tile;
+    int c = counts[row];
+    if (c < 0 || c > g.nT) {
+      if (lane == 0) set_status(status, kStatusBadBlock);
+      c = c < 0 ? 0 : g.nT;
+    }
+    const int* list = idx + row * (size_t)cap;
+    uint32_t* bmx = half ? bmb : bma;
+    for (int e = lane; e < c; e += 32) {
+      const int j = list[e];
+      const bool ok = j >= 0 && j < g.nT && (e == 0 || list[e - 1] < j);
+      if (!ok) {
+        set_status(status, kStatusBadBlock);
+        continue;
+      }
+      atomicOr(&bmx[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncwarp();
+  int* out = uni + item * (long long)g.nT;
+  int n = 0;
+  for (int w = 0; w < words; ++w) {
+    const int j = w * 32 + lane;
+    const uint32_t a = (bma[w] >> lane) & 1u, b = (bmb[w] >> lane) & 1u;
+    const uint32_t m = a | (b << 1);
+    const unsigned bal = __ballot_sync(0xffffffffu, m != 0u);
+    if (m) out[n + __popc(bal & ((1u << lane) - 1u))] = j | (int)(m << 16);
+    n += __popc(bal);
+  }
+  if (lane == 0) {
+    if (n == 0) {  // both rows empty: one fully masked step keeps the item well formed
+      out[0] = 0;
+      n = 1;
+    }
+    ucount[item] = n;
+  }
+}
+
+// rank(e) = #{e' : key(e') > key(e)} + #{e' < e : key(e') == key(e)};
+// worklist[rank(e)] = e.  Keys staged through shared memory in chunks.
+__global__ void __launch_bounds__(256) rank_kernel(const int* __restrict__ key, int n, int* __restrict__ worklist) {
+  __shared__ int ks[2048];
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int ke = e < n ? key[e] : 0;
+  int rank = 0;
+  for (int c0 = 0; c0 < n; c0 += 2048) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 2048 && c0 + i < n; i += blockDim.x) ks[i] = key[c0 + i];
+    __syncthreads();
+    const int lim = min(2048, n - c0);
+    for (int i = 0; i < lim; ++i) {
+      const int kk = ks[i];
+      rank += (kk > ke || (kk == ke && c0 + i < e)) ? 1 : 0;
+    }
+  }
+  if (e < n) worklist[rank] = e;
+}
+
+cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
+                         cudaStream_t s) {
+  const long long items = (long long)g.BH * g.P;
+  const int words = (g.nT + 31) / 32;
+  const size_t smem = (size_t)4 * 2 * words * sizeof(uint32_t);
+  union_kernel<<<(unsigned)((items + 3) / 4), 128, smem, s>>>(g, counts, idx, cap, uni, ucount, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rank(const int* key, int n, int* worklist, cudaStream_t s) {
+  rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(key, n, worklist);
+  return cudaGetLastError();
+}
+
+}  // namespace fvattn

@@ -1,0 +1,203 @@
+/*
+ * fvattn.h -- C ABI of libfvattn.so: adaptive block-sparse self-attention over
+ * 3D video latent tokens, for NVIDIA B200 (sm_100a).
+ *
+ * The path (pages: "VSA" digest, section 3; "FVAttn" digest, sections 00/02;
+ * "DFSAttn" digest, sections 1 and 3; "Causal-RoPE SP" digest, sections
+ * 2.2-2.3):
+ *   1. tokens of a T x Hg x W latent grid are grouped into 4x4x4 tiles
+ *      (64 tokens), in raster-cube or 3D Hilbert order;
+ *   2. optionally, a 3D rotary position encoding is applied to Q and K;
+ *   3. Q and K are mean-pooled per tile;
+ *   4. a coarse pooled Q K^T gives a softmax over key tiles per query tile;
+ *   5. per (batch, head, query tile) the key tiles are selected by top-p
+ *      cumulative mass with a k_min floor;
+ *   6. the fine stage runs softmax attention of each query token over the
+ *      tokens of its tile's selected key tiles only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors.  q, k, v, out are [B, H, N, d] row-major (d fastest), N = T*Hg*W;
+ *   lse is [B, H, N] float32.  dtype FVATTN_BF16 (bf16 storage, fp32
+ *   accumulation, bf16 tensor-core operands) or FVATTN_F32 (fp32 throughout).
+ *   Natural layout: token n = (t*Hg + h)*W + w.  Tiled layout: token rows
+ *   permuted so that tile j (in the chosen order) occupies rows 64j..64j+63,
+ *   as produced by fvattn_tile_reorder.  Tile ids always follow the order.
+ * Pointers.  Every tensor, block-list and workspace pointer is a DEVICE
+ *   pointer owned by the caller; the library never allocates or frees device
+ *   memory and keeps no pointer after a call returns.  Shapes, rope and
+ *   cache structs are HOST pointers read during the call.  Device pointers
+ *   must be 16-byte aligned; the workspace 256-byte aligned.
+ * Execution.  Calls enqueue kernels on the given stream and return without
+ *   synchronising (except fvattn_get_device_status).  Calls that share a
+ *   workspace must not overlap in time.
+ * Errors.  Argument, shape and capacity errors are detected on the host and
+ *   returned before anything is enqueued.  A failed launch returns
+ *   FVATTN_ERR_CUDA.  Errors found by a kernel (an out-of-range block index,
+ *   a wait that hit its iteration cap) set a status word in the workspace,
+ *   read with fvattn_get_device_status; kernels never trap.
+ * Limits.  grid extents multiples of the tile (4,4,4), each <= 4096;
+ *   d = 128 for BF16 (tensor-core fine stage), d in {32, 64, 128} for F32;
+ *   nT = N/64 <= 4096; B*H*N*d < 2^31.
+ */
+#ifndef FVATTN_H
+#define FVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fvattn_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  FVATTN_OK = 0,
+  FVATTN_ERR_INVALID_ARG = -1,     /* null pointer, bad enum, top_p NaN, misaligned pointer */
+  FVATTN_ERR_SHAPE = -2,           /* grid not a multiple of the tile, bad head_dim, too large */
+  FVATTN_ERR_DTYPE = -3,
+  FVATTN_ERR_CAPACITY = -4,        /* blocks.cap < nT */
+  FVATTN_ERR_CUDA = -5,            /* a CUDA runtime/driver call failed */
+  FVATTN_ERR_CACHE_MISMATCH = -6,  /* reuse_mask with a cache filled for another shape */
+  FVATTN_ERR_DEVICE = -7,          /* a kernel set the device status word */
+  FVATTN_ERR_WORKSPACE = -8,       /* ws_bytes smaller than fvattn_workspace_size */
+  FVATTN_ERR_UNSUPPORTED = -9      /* device is not sm_100, or a combination not built */
+} fvattn_status;
+
+typedef enum { FVATTN_F32 = 0, FVATTN_BF16 = 1 } fvattn_dtype;
+typedef enum { FVATTN_ORDER_RASTER_CUBE = 0, FVATTN_ORDER_HILBERT = 1 } fvattn_order;
+typedef enum { FVATTN_LAYOUT_NATURAL = 0, FVATTN_LAYOUT_TILED = 1 } fvattn_layout;
+
+typedef struct { int32_t T, H, W; } fvattn_dims;   /* latent grid (frames, height, width) */
+typedef struct { int32_t t, h, w; } fvattn_tile;   /* tile edge per axis; only 4,4,4 is supported */
+
+/* 3D rotary encoding ("Causal-RoPE SP" digest, sections 2.2-2.3): head dims
+ * split into groups of dt, dh, dw (dt+dh+dw == d, each even) for the t, h,
+ * w axes; in a group of size da, dims (2j, 2j+1) rotate by pos*base^(-2j/da),
+ * pos the token's integer grid coordinate on that axis.  Pooling uses the
+ * rotated values in fp32; the fine stage uses them rounded to the dtype. */
+typedef struct { int32_t enabled, dt, dh, dw; float base; } fvattn_rope;
+
+typedef struct {
+  int32_t batch, heads, head_dim;
+  fvattn_dims grid;
+  fvattn_tile tile;
+  fvattn_dtype dtype;
+  fvattn_order order;
+  fvattn_layout layout;   /* layout of q, k, v, out, lse in pool_select / block_sparse_fwd */
+  float scale;            /* softmax scale for coarse and fine logits; 0 => 1/sqrt(head_dim) */
+} fvattn_shape;
+
+/* Selected key tiles per (batch, head, query tile).  counts [B,H,nT] int32;
+ * idx [B,H,nT,cap] int32 with row r's first counts[r] entries the selected
+ * tile ids in ascending order; entries past counts[r] are not written and
+ * not read.  cap >= nT. */
+typedef struct { int32_t* counts; int32_t* idx; int32_t cap; } fvattn_blocks;
+
+/* Block lists kept across diffusion steps ("DFSAttn" digest, section 3).
+ * blocks are caller-owned device buffers; shape/top_p/k_min/valid are
+ * written by fvattn_forward when it fills the cache. */
+typedef struct {
+  fvattn_blocks blocks;
+  fvattn_shape shape;
+  float top_p;
+  int32_t k_min;
+  int32_t valid;
+} fvattn_mask_cache;
+
+/* nT = N / 64 for a valid shape. */
+int fvattn_num_tiles(const fvattn_shape* shape, int64_t* num_tiles);
+
+/* Bytes of device workspace every entry point below needs for this shape
+ * (the maximum over them, rope included when rope != NULL && rope->enabled). */
+int fvattn_workspace_size(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes);
+
+/* Step 1 ("VSA" digest, section 3: (4,4,4) cubes; "DFSAttn" digest,
+ * section 1: Hilbert reordering before blocking).  Permutes token rows of a
+ * [B*H, N, row_bytes] tensor between natural and tiled layout:
+ * inverse == 0: y[pi(n)] = x[n]; inverse != 0: y[n] = x[pi(n)], where pi(n)
+ * is token n's tiled position in shape->order.  row_bytes is a multiple of 4
+ * in [4, 1024] (d*sizeof(dtype) for q/k/v/out, 4 for lse).  x and y must not
+ * overlap.  shape->layout is ignored. */
+int fvattn_tile_reorder(const fvattn_shape* shape, const void* x, void* y, int32_t row_bytes,
+                        int inverse, void* ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Steps 2-5 ("VSA" digest, section 3: pooled coarse stage predicting tile
+ * importance; "FVAttn" digest, sections 00/02: top-p routing with a top-k
+ * floor).  q, k in shape->layout.  Writes out->counts and out->idx.
+ * count = min(nT, max(m, k_min)), m >= 1 the fewest tiles whose coarse
+ * softmax mass reaches top_p (ties to the lower tile id); top_p >= 1 keeps
+ * every tile; top_p <= 0 with k_min = k is fixed top-k.  rope may be NULL. */
+int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k,
+                       const fvattn_rope* rope, float top_p, int32_t k_min,
+                       const fvattn_blocks* out, void* ws, size_t ws_bytes,
+                       fvattn_stream_t stream);
+
+/* Schedule of the fine stage (single-GPU analogue of the "FVAttn" digest's
+ * runtime head-level load balancing, section 02): work items are pairs of
+ * adjacent query tiles (2p, 2p+1) of one (batch, head), encoded
+ * ((b*H + h)*P + p) with P = ceil(nT/2); the cost of an item is the size of
+ * the union of the two tiles' lists (the single tile's list for the last
+ * item of an odd nT); items are sorted by cost descending, ties by ascending
+ * item code (longest-processing-time first).  worklist has B*H*P int32. */
+int fvattn_build_worklist(const fvattn_shape* shape, const fvattn_blocks* blocks,
+                          int32_t* worklist, void* ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Step 6 ("VSA" digest, section 3: token-level attention inside the selected
+ * tiles; "CalibAtt" digest: selected connections computed densely, the rest
+ * skipped).  q, k, v, out, lse in shape->layout; out has the input dtype,
+ * lse is the natural-log softmax normaliser.  With rope enabled q and k are
+ * rotated first.  Block ids are checked on the device (bad ids set the
+ * status word and the row's output is left unwritten). */
+int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void* k,
+                            const void* v, const fvattn_rope* rope, const fvattn_blocks* blocks,
+                            void* out, float* lse, void* ws, size_t ws_bytes,
+                            fvattn_stream_t stream);
+
+/* The whole path on natural-layout tensors (shape->layout is ignored).
+ * cache == NULL: select and attend.  cache != NULL, reuse_mask == 0: select,
+ * store the lists into cache->blocks and stamp the cache.  reuse_mask != 0:
+ * skip steps 2-5 and attend with cache->blocks ("DFSAttn" digest, section 3);
+ * returns FVATTN_ERR_CACHE_MISMATCH if the cache is not valid for this shape. */
+int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, const void* v,
+                   const fvattn_rope* rope, float top_p, int32_t k_min, fvattn_mask_cache* cache,
+                   int reuse_mask, void* out, float* lse, void* ws, size_t ws_bytes,
+                   fvattn_stream_t stream);
+
+/* Synchronises the stream, reads and clears the workspace status word.
+ * *status is 0 or a positive code: 1 bad block id, 2 wait cap reached. */
+int fvattn_get_device_status(void* ws, fvattn_stream_t stream, int32_t* status);
+
+/* Failure-detection self test: launches one block that waits, with the
+ * library's bounded wait, on a barrier nothing ever completes, using the
+ * given iteration cap.  The kernel gives up, sets status 2 in the workspace
+ * status word and returns; read it with fvattn_get_device_status. */
+int fvattn_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t cap_iterations,
+                                 fvattn_stream_t stream);
+
+/* Per-stage timing.  While enabled, every entry point records a pair of CUDA
+ * events on its stream around each kernel it launches (host-side event
+ * objects only; no device memory).  fvattn_profile_read synchronises on the
+ * recorded events, writes the summed milliseconds and launch counts per
+ * stage into ms[FVATTN_STAGE_COUNT] and launches[FVATTN_STAGE_COUNT]
+ * (either may be NULL) and clears the record.  Not thread-safe against
+ * concurrent calls from several host threads. */
+typedef enum {
+  FVATTN_STAGE_TABLES = 0,    /* tile / token / RoPE tables */
+  FVATTN_STAGE_REORDER = 1,   /* fvattn_tile_reorder */
+  FVATTN_STAGE_POOL = 2,      /* pooling (+ RoPE, rotated copies) */
+  FVATTN_STAGE_SELECT = 3,    /* coarse scores, softmax, top-p selection */
+  FVATTN_STAGE_SCHEDULE = 4,  /* union lists + work-list sort */
+  FVATTN_STAGE_FINE = 5,      /* block-sparse fine attention */
+  FVATTN_STAGE_COUNT = 6
+} fvattn_stage;
+int fvattn_profile_enable(int enable);
+int fvattn_profile_read(double* ms, int64_t* launches);
+
+const char* fvattn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FVATTN_H */
