@@ -1,0 +1,61 @@
+// fvattn_pool_select_noalloc: the pool/select step for callers that cannot
+// allocate device memory.
+//
+// Some callers have no way to obtain a workspace buffer: a plugin running
+// inside a host application that owns every device allocation and hands the
+// plugin only its input and output tensors, or code on a latency-critical
+// path where the device-wide synchronisation of cudaMalloc is not allowed.
+// For them this entry point runs the same kernels as fvattn_pool_select with
+// its scratch memory (tile tables, pooled Q/K) in one statically sized
+// device array that is part of this library.  The caller still provides
+// q, k and the block-list buffers.
+//
+// The array below is a host-side name only: its device address is looked up
+// with cudaGetSymbolAddress the first time the entry point runs on each
+// device (with that device current) and cached; kernels only ever receive
+// that address.
+#include <mutex>
+
+#include "fvattn_internal.cuh"
+
+// 32 MiB.  A shape is accepted when its full workspace
+// (fvattn_workspace_size) fits: for example the 16x32x32 latent with 12
+// heads (7.6 MiB) or the 20x32x52 latent with up to 8 heads (16.6 MiB); the
+// 20x32x52 latent with 40 heads (82.5 MiB) is rejected.
+static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+
+static __device__ __align__(256) unsigned char g_pool_select_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FVATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pool_select_scratch) != cudaSuccess || !p) return FVATTN_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FVATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void* q, const void* k,
+                                          const fvattn_rope* rope, float top_p, int32_t k_min,
+                                          const fvattn_blocks* out, fvattn_stream_t stream) {
+  size_t need = 0;
+  const int st = fvattn_workspace_size(shape, rope, &need);
+  if (st != FVATTN_OK) return st;
+  if (need > kNoAllocScratchBytes) return FVATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int sa = scratch_address(&scratch);
+  if (sa != FVATTN_OK) return sa;
+  return fvattn_pool_select(shape, q, k, rope, top_p, k_min, out, scratch, kNoAllocScratchBytes, stream);
+}

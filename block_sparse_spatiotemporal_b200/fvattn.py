@@ -21,7 +21,7 @@ __all__ = [
     "make_shape", "make_rope", "num_tiles", "workspace_size", "workspace",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
-    "STAGES",
+    "STAGES", "pool_select_noalloc",
 ]
 
 F32, BF16 = 0, 1
@@ -80,6 +80,8 @@ _SIGS = {
     "fvattn_pool_select": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
                            ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p,
                            ctypes.c_size_t, ctypes.c_void_p],
+    "fvattn_pool_select_noalloc": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
+                                   ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p],
     "fvattn_build_worklist": [ctypes.POINTER(Shape), ctypes.POINTER(Blocks), ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_block_sparse_fwd": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -202,6 +204,20 @@ def pool_select(shape: Shape, q, k, ws, top_p: float, k_min: int, rope: Optional
     _check("fvattn_pool_select", lib().fvattn_pool_select(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope),
                                                           float(top_p), int(k_min), ctypes.byref(b), _ptr(ws),
                                                           ws.numel(), _stream(stream)))
+    return counts, idx
+
+
+def pool_select_noalloc(shape: Shape, q, k, top_p: float, k_min: int, rope: Optional[Rope] = None, blocks=None,
+                        stream=None):
+    """Steps 2-5 with the library's static scratch instead of a workspace
+    (for callers that cannot allocate); returns (counts, idx)."""
+    if blocks is None:
+        counts, idx, b = new_blocks(shape, q.device)
+    else:
+        counts, idx, b = blocks
+    _check("fvattn_pool_select_noalloc",
+           lib().fvattn_pool_select_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope), float(top_p),
+                                            int(k_min), ctypes.byref(b), _stream(stream)))
     return counts, idx
 
 

@@ -134,6 +134,26 @@ int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k,
                        const fvattn_blocks* out, void* ws, size_t ws_bytes,
                        fvattn_stream_t stream);
 
+/* Steps 2-5 without a caller workspace.  The pages have no counterpart:
+ * this is for callers that cannot allocate device memory (a plugin whose
+ * host application owns every device allocation and passes in only the
+ * input and output tensors, or code on a latency-critical path where the
+ * device-wide synchronisation of cudaMalloc is not allowed).  Arguments,
+ * layout and results are those of fvattn_pool_select; the scratch memory
+ * is a 32 MiB array inside the library that every GPU loading the library
+ * holds until the process exits.  Shapes whose workspace
+ * (fvattn_workspace_size) exceeds 32 MiB are rejected with
+ * FVATTN_ERR_WORKSPACE before anything is enqueued.  No call allocates
+ * memory.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents (each call rewrites every part it reads),
+ * so calls that overlap on the GPU (other streams, other host threads)
+ * race: serialise them. */
+int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void* q, const void* k,
+                               const fvattn_rope* rope, float top_p, int32_t k_min,
+                               const fvattn_blocks* out, fvattn_stream_t stream);
+
 /* Schedule of the fine stage (single-GPU analogue of the "FVAttn" digest's
  * runtime head-level load balancing, section 02): work items are pairs of
  * adjacent query tiles (2p, 2p+1) of one (batch, head), encoded
