@@ -29,8 +29,10 @@ Readings where the pages are silent (each also listed in the design notes):
   * coarse logits are scale * Qp . Kp with scale = 1/sqrt(d); normalisation is
     a softmax over the key tiles of each query-tile row;
   * top-p keeps the fewest tiles (at least one) whose cumulative mass, summed
-    in descending order, reaches p (``>= p``); ties go to the lower tile
-    index; count = min(nT, max(m, k_min)); p >= 1 keeps every tile;
+    in descending order, reaches p (``>= p``); tiles are ranked by their
+    coarse logit (the probability order, without the ties that underflowing
+    probabilities would create), ties to the lower tile index;
+    count = min(nT, max(m, k_min)); p >= 1 keeps every tile;
   * the output is the fine stage only (the coarse stage only routes);
   * lse is the natural log of the softmax normaliser;
   * RoPE: per-axis groups of 44/42/42 head dims for (t, h, w), adjacent pairs
@@ -215,25 +217,40 @@ def pool_tiles(x_tiled, tile_tokens=64):
     return np.asarray(x_tiled, np.float64).reshape(N // tile_tokens, tile_tokens, d).mean(axis=1)
 
 
-def coarse_probabilities(qp, kp, scale):
-    """Row softmax of the pooled logits scale * Qp Kp^T: [nT, nT]."""
-    s = scale * (qp @ kp.T)
-    s = s - s.max(axis=1, keepdims=True)
+def coarse_logits(qp, kp, scale):
+    """Pooled coarse logits scale * Qp Kp^T: [nT, nT]."""
+    return scale * (qp @ kp.T)
+
+
+def row_softmax(S):
+    s = S - S.max(axis=1, keepdims=True)
     e = np.exp(s)
     return e / e.sum(axis=1, keepdims=True)
+
+
+def coarse_probabilities(qp, kp, scale):
+    """Row softmax of the pooled logits scale * Qp Kp^T: [nT, nT]."""
+    return row_softmax(coarse_logits(qp, kp, scale))
 
 
 BORDER = 1e-5
 
 
-def select_blocks(P, top_p, k_min):
-    """Top-p selection with a k_min floor for each row of P [nT, nT].
+def select_blocks(S, top_p, k_min):
+    """Top-p selection with a k_min floor for each row of the coarse logits
+    S [nT, nT] (probabilities P = row softmax of S).
+
+    Tiles are ranked by probability, descending, ties to the lower tile id.
+    The ranking is taken on the logits: softmax is monotone in the logit, so
+    the order is the same, but tiles whose probability underflows to zero
+    keep their true order instead of becoming spurious ties.
 
     Returns counts [nT], idx [nT, nT] (ascending tile ids, -1 padded) and
     a boolean [nT] marking borderline rows, whose count could change if the
     cumulative masses moved by 1e-5."""
+    P = row_softmax(S)
     nT = P.shape[1]
-    order = np.argsort(-P, axis=1, kind="stable")       # desc, ties -> lower id
+    order = np.argsort(-S, axis=1, kind="stable")       # desc, ties -> lower id
     cum = np.cumsum(np.take_along_axis(P, order, axis=1), axis=1)
 
     def count_for(p):
@@ -254,16 +271,16 @@ def select_blocks(P, top_p, k_min):
     return counts, idx, border
 
 
-def near_tie_rows(P, counts, rel=1e-6):
-    """Rows whose last kept and first dropped probabilities are within rel."""
-    nT = P.shape[1]
-    srt = -np.sort(-P, axis=1)
-    out = np.zeros(P.shape[0], bool)
-    for r in range(P.shape[0]):
+def near_tie_rows(S, counts, tol):
+    """Rows whose last kept and first dropped logits differ by at most
+    tol[r] (the rounding error a float32 evaluation of the row may carry)."""
+    nT = S.shape[1]
+    srt = -np.sort(-S, axis=1)
+    out = np.zeros(S.shape[0], bool)
+    for r in range(S.shape[0]):
         c = counts[r]
         if 0 < c < nT:
-            a, b = srt[r, c - 1], srt[r, c]
-            out[r] = abs(a - b) <= rel * max(abs(a), 1e-300)
+            out[r] = srt[r, c - 1] - srt[r, c] <= tol[r]
     return out
 
 
@@ -331,10 +348,12 @@ def coarse_head(q, k, grid, order, top_p, k_min, scale, rope=None, pos=None):
         k = rope_3d(k, coords, rope["dims"], rope["base"])
     qt, kt = to_tiled(q, pos), to_tiled(k, pos)
     qp, kp = pool_tiles(qt), pool_tiles(kt)
-    P = coarse_probabilities(qp, kp, scale)
-    counts, idx, border = select_blocks(P, top_p, k_min)
-    return dict(q_tiled=qt, k_tiled=kt, qp=qp, kp=kp, P=P, counts=counts,
-                idx=idx, border=border, pos=pos)
+    S = coarse_logits(qp, kp, scale)
+    counts, idx, border = select_blocks(S, top_p, k_min)
+    # magnitude of the terms of each logit: scale * |Qp| . |Kp|
+    s_abs = scale * (np.abs(qp) @ np.abs(kp).T)
+    return dict(q_tiled=qt, k_tiled=kt, qp=qp, kp=kp, S=S, P=row_softmax(S), s_abs=s_abs,
+                counts=counts, idx=idx, border=border, pos=pos)
 
 
 def forward_head(q, k, v, grid, order, top_p, k_min, dtype, scale=None,

@@ -139,7 +139,7 @@ def test_select_matches_brute_force_over_subsets(seed):
     P = rng.dirichlet(np.full(nT, 0.5), size=6)
     for p in (0.0, 0.3, 0.5, 0.8, 0.9, 0.95, 0.99, 1.0):
         for k_min in (0, 1, 2, 4, 12):
-            counts, idx, border = O.select_blocks(P, p, k_min)
+            counts, idx, border = O.select_blocks(np.log(P), p, k_min)
             for r in range(P.shape[0]):
                 c = counts[r]
                 assert c == _brute_force_count(P[r], p, k_min), (p, k_min, r)
@@ -156,20 +156,34 @@ def test_select_matches_brute_force_over_subsets(seed):
 
 def test_select_ties_go_to_lower_index_and_fixed_topk():
     P = np.array([[0.25, 0.25, 0.25, 0.25], [0.1, 0.4, 0.1, 0.4]])
-    counts, idx, _ = O.select_blocks(P, 0.5, 1)
+    counts, idx, _ = O.select_blocks(np.log(P), 0.5, 1)
     assert counts.tolist() == [2, 2]
     assert idx[0, :2].tolist() == [0, 1] and idx[1, :2].tolist() == [1, 3]
-    counts, idx, _ = O.select_blocks(P, 0.0, 3)
+    counts, idx, _ = O.select_blocks(np.log(P), 0.0, 3)
     assert counts.tolist() == [3, 3]
     assert idx[0, :3].tolist() == [0, 1, 2] and idx[1, :3].tolist() == [0, 1, 3]
 
 
+def test_select_ranks_underflowing_tiles_by_logit():
+    """Probabilities exp(-900) and exp(-800) are both 0.0 in float64, yet the
+    tile with the larger logit is the more probable one and ranks first."""
+    S = np.array([[0.0, -900.0, -800.0, -5.0]])
+    P = O.row_softmax(S)
+    assert P[0, 1] == 0.0 and P[0, 2] == 0.0
+    counts, idx, _ = O.select_blocks(S, 0.0, 3)
+    assert counts.tolist() == [3] and idx[0, :3].tolist() == [0, 2, 3]
+    assert O.near_tie_rows(S, counts, np.array([1e-3])).tolist() == [False]
+    S2 = np.array([[0.0, -900.0, -5.0 - 1e-7, -5.0]])
+    c2, _, _ = O.select_blocks(S2, 0.0, 2)
+    assert O.near_tie_rows(S2, c2, np.array([1e-6])).tolist() == [True]
+
+
 def test_select_borderline_flag():
     P = np.array([[0.6, 0.3, 0.1], [0.5, 0.3 + 4e-6, 0.2 - 4e-6]])
-    _, _, border = O.select_blocks(P, 0.8, 1)
+    _, _, border = O.select_blocks(np.log(P), 0.8, 1)
     assert border.tolist() == [False, True]
     # with a k_min floor above both candidate counts the row is not borderline
-    _, _, border = O.select_blocks(P, 0.8, 3)
+    _, _, border = O.select_blocks(np.log(P), 0.8, 3)
     assert border.tolist() == [False, False]
 
 
