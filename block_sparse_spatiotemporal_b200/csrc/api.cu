@@ -99,6 +99,7 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r) {
   L.uni = take(sizeof(int) * (size_t)g.BH * g.P * g.nT);
   L.ucount = take(sizeof(int) * (size_t)g.BH * g.P);
   L.worklist = take(sizeof(int) * (size_t)g.BH * g.P);
+  L.rank = take(sizeof(int) * (size_t)g.BH * g.P);
   const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
   L.qrot = take(rot);
   L.krot = take(rot);
@@ -292,7 +293,7 @@ int run_schedule(const Call& c, const fvattn_blocks* blocks, int* worklist) {
   StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
   FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
                        c.status, c.s));
-  FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, worklist, c.s));
+  FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, c.at<int>(c.L.rank), worklist, c.s));
   return FVATTN_OK;
 }
 

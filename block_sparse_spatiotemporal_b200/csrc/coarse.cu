@@ -172,10 +172,19 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
 }
 
 // --------------------------------------------------------------------------
-// Score + select.  Block = 8 warps handling R = 8*RPW consecutive query tiles
-// of one head.  Phase 1 computes S[R][nT] = scale * Qp Kp^T in shared memory
-// (fp32 FFMA, register-tiled: each thread RPW rows x 2 key tiles).  Phase 2:
-// warp w selects rows w*RPW .. w*RPW+RPW-1.
+// Score + select.  Block = 16 warps handling R <= 32 consecutive query tiles
+// of one head.  Phase 1 computes S[R][nT] = scale * Qp Kp^T (fp32 FFMA) into
+// shared memory.  Phase 2: warp w selects rows w and w + 16.
+//
+// Tiles are ranked by their logit (the probability order; exp(s - max)
+// underflows to 0 for distant tiles, the logit does not), descending, ties
+// to the lower tile id.  A row's logits sit in registers, lane-strided
+// (element i of a lane is tile 32 i + lane).  Most rows are settled by a few
+// argmax rounds that pick tiles in rank order and add their probabilities in
+// that order until the cut and the k_min floor are both reached.  Rows whose
+// cut lies deeper use a bisection over the 32-bit order-preserving keys of
+// the logits: the largest key u whose suffix mass sum_{key >= u} e reaches
+// top_p * Z (warp-tree sums), then ties at u are taken lowest id first.
 // --------------------------------------------------------------------------
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -193,16 +202,209 @@ __device__ inline int warp_isum(int v) {
   return v;
 }
 
-constexpr int kKC = 64;   // key tiles per phase-1 chunk
-constexpr int kKCS = 66;  // padded chunk row stride (floats)
+// Unsigned key with the order of the float (no NaNs expected).
+__device__ inline uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
 
-template <int RPW, int D>
-__global__ void __launch_bounds__(256) select_kernel(Geom g, const float* __restrict__ qp,
-                                                     const float* __restrict__ kp, float top_p, int k_min,
-                                                     int* __restrict__ counts, int* __restrict__ idx, int cap) {
-  constexpr int R = 8 * RPW;
+constexpr int kKC = 64;          // key tiles per phase-1 chunk
+constexpr int kKCS = 66;         // padded chunk row stride (floats)
+constexpr int kMaxRounds = 32;   // argmax rounds before falling back to bisection
+
+// Selection of one row; srow holds the row's nT logits on entry and the
+// probabilities' numerators e_j = exp(s_j - max) on exit.
+template <int MAXV>
+__device__ void select_row(float* srow, int nT, float top_p, int k_min, int* count_out, int* list) {
+  constexpr int NW = (MAXV + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  float v[MAXV];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int j = i * 32 + lane;
+    v[i] = j < nT ? srow[j] : -INFINITY;
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) mx = fmaxf(mx, v[i]);
+  mx = warp_max(mx);
+  float zp = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int j = i * 32 + lane;
+    if (j < nT) {
+      const float e = expf(v[i] - mx);
+      srow[j] = e;
+      zp += e;
+    }
+  }
+  const float Z = warp_sum(zp);
+  __syncwarp();
+
+  if (top_p >= 1.0f) {
+    for (int j = lane; j < nT; j += 32) list[j] = j;
+    if (lane == 0) *count_out = nT;
+    return;
+  }
+  const float target = top_p * Z;
+  const int floor_k = k_min > 1 ? k_min : 1;
+
+  // ---- argmax rounds
+  uint32_t tk[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) tk[w] = 0u;
+  int m = top_p > 0.f ? 0 : 1;
+  int count = m ? (floor_k < nT ? floor_k : nT) : -1;
+  int picks = 0;
+  float cum = 0.f;
+  const int rounds = (floor_k > kMaxRounds) ? 0 : (nT < kMaxRounds ? nT : kMaxRounds);
+  for (int r = 0; r < rounds; ++r) {
+    if (count >= 0 && picks >= count) break;
+    float bv = -INFINITY;
+    int bj = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const bool free_i = !((tk[i >> 5] >> (i & 31)) & 1u);
+      if (free_i && v[i] > bv) {
+        bv = v[i];
+        bj = i * 32 + lane;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (ov > bv || (ov == bv && oj < bj)) {
+        bv = ov;
+        bj = oj;
+      }
+    }
+    if (bj == 0x7fffffff) break;
+    if ((bj & 31) == lane) {
+      const int i = bj >> 5;
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        if (w == (i >> 5)) tk[w] |= 1u << (i & 31);
+    }
+    cum += srow[bj];
+    ++picks;
+    if (m == 0 && cum >= target) m = picks;
+    if (m > 0 && count < 0) {
+      count = m > floor_k ? m : floor_k;
+      if (count > nT) count = nT;
+    }
+  }
+
+  int* out = list;
+  if (count >= 0 && picks >= count) {
+    int base = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const bool sel = (tk[i >> 5] >> (i & 31)) & 1u;
+      const unsigned b = __ballot_sync(0xffffffffu, sel);
+      if (sel) out[base + __popc(b & ((1u << lane) - 1u))] = i * 32 + lane;
+      base += __popc(b);
+    }
+    if (lane == 0) *count_out = count;
+    return;
+  }
+
+  // ---- bisection over the keys
+  uint32_t uT = 0;
+  int take = 0;
+  if (m == 0) {
+    uint32_t u = 0;
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t cand = u | (1u << b);
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i) {
+        const int j = i * 32 + lane;
+        part += (j < nT && order_key(v[i]) >= cand) ? srow[j] : 0.f;
+      }
+      if (warp_sum(part) >= target) u = cand;
+    }
+    float gpart = 0.f;
+    int cgt = 0, ceq = 0;
+    float eu = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int j = i * 32 + lane;
+      if (j < nT) {
+        const uint32_t kk = order_key(v[i]);
+        if (kk > u) {
+          gpart += srow[j];
+          ++cgt;
+        } else if (kk == u) {
+          ++ceq;
+          eu = srow[j];
+        }
+      }
+    }
+    const float mgt = warp_sum(gpart);
+    cgt = warp_isum(cgt);
+    ceq = warp_isum(ceq);
+    eu = warp_max(eu);
+    int r_ties = 0;
+    if (ceq > 0) {
+      float accm = mgt + eu;
+      r_ties = 1;
+      while (r_ties < ceq && accm < target) {
+        accm += eu;
+        ++r_ties;
+      }
+    }
+    m = cgt + r_ties;
+    if (m < 1) m = 1;
+    count = m > floor_k ? m : floor_k;
+    if (count > nT) count = nT;
+    if (count == m) {
+      uT = u;
+      take = r_ties;
+    }
+  }
+  if (take == 0 && !(count == m && m > 0 && uT != 0)) {
+    // top-`count` set: largest key u2 with #{key >= u2} >= count
+    uint32_t u2 = 0;
+    for (int b = 31; b >= 0; --b) {
+      const uint32_t cand = u2 | (1u << b);
+      int c = 0;
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i) c += (i * 32 + lane < nT && order_key(v[i]) >= cand) ? 1 : 0;
+      if (warp_isum(c) >= count) u2 = cand;
+    }
+    int cgt = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) cgt += (i * 32 + lane < nT && order_key(v[i]) > u2) ? 1 : 0;
+    cgt = warp_isum(cgt);
+    uT = u2;
+    take = count - cgt;
+  }
+  int base = 0, tie_base = 0;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int j = i * 32 + lane;
+    const uint32_t kk = j < nT ? order_key(v[i]) : 0u;
+    const bool tie = j < nT && kk == uT;
+    const unsigned tmask = __ballot_sync(0xffffffffu, tie);
+    const int trank = tie_base + __popc(tmask & ((1u << lane) - 1u));
+    const bool sel = j < nT && (kk > uT || (tie && trank < take));
+    const unsigned smask = __ballot_sync(0xffffffffu, sel);
+    const int pos = base + __popc(smask & ((1u << lane) - 1u));
+    if (sel && pos < count) out[pos] = j;
+    base += __popc(smask);
+    tie_base += __popc(tmask);
+  }
+  if (lane == 0) *count_out = count;
+}
+
+template <int D, int MAXV, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) select_kernel(Geom g, const float* __restrict__ qp,
+                                                            const float* __restrict__ kp, float top_p, int k_min,
+                                                            int* __restrict__ counts, int* __restrict__ idx, int cap,
+                                                            int R) {
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                       // [D][R]   transposed query rows
+  float* qs = sm;                       // [D][R]    transposed query rows
   float* ks = qs + D * R;               // [D][kKCS] transposed key chunk
   float* S = ks + D * kKCS;             // [R][nT]
   const int nT = g.nT;
@@ -216,6 +418,7 @@ __global__ void __launch_bounds__(256) select_kernel(Geom g, const float* __rest
     const int r = i / D, c = i % D;
     qs[c * R + r] = (row0 + r < nT) ? qph[(size_t)(row0 + r) * D + c] : 0.f;
   }
+  const bool two = R > WARPS;                     // rows warp and warp + WARPS
   for (int kc = 0; kc < nT; kc += kKC) {
     __syncthreads();
     for (int i = threadIdx.x; i < D * kKC; i += blockDim.x) {
@@ -223,132 +426,36 @@ __global__ void __launch_bounds__(256) select_kernel(Geom g, const float* __rest
       ks[c * kKCS + kk] = (kc + kk < nT) ? kph[(size_t)(kc + kk) * D + c] : 0.f;
     }
     __syncthreads();
-    float acc[RPW][2];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) acc[r][0] = acc[r][1] = 0.f;
+    if (warp < R) {
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
 #pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-      const float2 kv = *reinterpret_cast<const float2*>(&ks[c * kKCS + 2 * lane]);
-      float qv[RPW];
-      if constexpr (RPW == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(&qs[c * R + warp * 4]);
-        qv[0] = t.x; qv[1] = t.y; qv[2] = t.z; qv[3] = t.w;
-      } else {
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) qv[r] = qs[c * R + warp * RPW + r];
+      for (int c = 0; c < D; ++c) {
+        const float2 kv = *reinterpret_cast<const float2*>(&ks[c * kKCS + 2 * lane]);
+        const float q0 = qs[c * R + warp];
+        a00 = fmaf(q0, kv.x, a00);
+        a01 = fmaf(q0, kv.y, a01);
+        if (two) {
+          const float q1 = qs[c * R + warp + WARPS];
+          a10 = fmaf(q1, kv.x, a10);
+          a11 = fmaf(q1, kv.y, a11);
+        }
       }
-#pragma unroll
-      for (int r = 0; r < RPW; ++r) {
-        acc[r][0] = fmaf(qv[r], kv.x, acc[r][0]);
-        acc[r][1] = fmaf(qv[r], kv.y, acc[r][1]);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
       const int kk = kc + 2 * lane;
-      if (kk < nT) S[(warp * RPW + r) * nT + kk] = acc[r][0] * g.scale;
-      if (kk + 1 < nT) S[(warp * RPW + r) * nT + kk + 1] = acc[r][1] * g.scale;
+      if (kk < nT) S[warp * nT + kk] = a00 * g.scale;
+      if (kk + 1 < nT) S[warp * nT + kk + 1] = a01 * g.scale;
+      if (two) {
+        if (kk < nT) S[(warp + WARPS) * nT + kk] = a10 * g.scale;
+        if (kk + 1 < nT) S[(warp + WARPS) * nT + kk + 1] = a11 * g.scale;
+      }
     }
   }
   __syncthreads();
 
-  for (int rr = 0; rr < RPW; ++rr) {
-    const int lr = warp * RPW + rr;
+  for (int lr = warp; lr < R; lr += WARPS) {
     const int row = row0 + lr;
     if (row >= nT) break;
-    float* s = S + lr * nT;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(s);
-    float mx = -INFINITY;
-    for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, s[j]);
-    mx = warp_max(mx);
-    float zpart = 0.f;
-    for (int j = lane; j < nT; j += 32) {
-      const float e = expf(s[j] - mx);
-      s[j] = e;
-      zpart += e;
-    }
-    const float Z = warp_sum(zpart);
-    __syncwarp();
-
-    int count;
-    uint32_t uT = 0;       // threshold bit pattern of the selected set
-    int take = 0;          // tiles with bits == uT to take, lowest ids first
-    if (top_p >= 1.0f) {
-      count = nT;
-    } else {
-      int m = 1;
-      uint32_t u = 0;
-      int r_ties = 1;
-      if (top_p > 0.f) {
-        const float target = top_p * Z;
-        for (int b = 29; b >= 0; --b) {
-          const uint32_t cand = u | (1u << b);
-          float part = 0.f;
-          for (int j = lane; j < nT; j += 32) part += bits[j] >= cand ? s[j] : 0.f;
-          if (warp_sum(part) >= target) u = cand;
-        }
-        float gpart = 0.f;
-        int cgt = 0, ceq = 0;
-        for (int j = lane; j < nT; j += 32) {
-          gpart += bits[j] > u ? s[j] : 0.f;
-          cgt += bits[j] > u ? 1 : 0;
-          ceq += bits[j] == u ? 1 : 0;
-        }
-        const float mgt = warp_sum(gpart);
-        cgt = warp_isum(cgt);
-        ceq = warp_isum(ceq);
-        const float eu = __uint_as_float(u);
-        float accm = mgt + eu;
-        r_ties = 1;
-        while (r_ties < ceq && accm < target) {
-          accm += eu;
-          ++r_ties;
-        }
-        m = ceq > 0 ? cgt + r_ties : (cgt > 0 ? cgt : 1);
-        if (ceq == 0) r_ties = 0;
-      }
-      count = m > k_min ? m : k_min;
-      if (count > nT) count = nT;
-      if (count == m && top_p > 0.f) {
-        uT = u;
-        take = r_ties;
-      } else {
-        // top-`count` set: largest u2 with #{bits >= u2} >= count
-        uint32_t u2 = 0;
-        for (int b = 30; b >= 0; --b) {
-          const uint32_t cand = u2 | (1u << b);
-          int c = 0;
-          for (int j = lane; j < nT; j += 32) c += bits[j] >= cand ? 1 : 0;
-          if (warp_isum(c) >= count) u2 = cand;
-        }
-        int cgt = 0;
-        for (int j = lane; j < nT; j += 32) cgt += bits[j] > u2 ? 1 : 0;
-        cgt = warp_isum(cgt);
-        uT = u2;
-        take = count - cgt;
-      }
-    }
-
-    int* out = idx + ((size_t)bh * nT + row) * (size_t)cap;
-    if (count == nT) {
-      for (int j = lane; j < nT; j += 32) out[j] = j;
-    } else {
-      int base = 0, tie_base = 0;
-      for (int j0 = 0; j0 < nT; j0 += 32) {
-        const int j = j0 + lane;
-        const uint32_t bj = j < nT ? bits[j] : 0u;
-        const bool tie = j < nT && bj == uT;
-        const unsigned tmask = __ballot_sync(0xffffffffu, tie);
-        const int trank = tie_base + __popc(tmask & ((1u << lane) - 1u));
-        const bool sel = j < nT && (bj > uT || (tie && trank < take));
-        const unsigned smask = __ballot_sync(0xffffffffu, sel);
-        const int pos = base + __popc(smask & ((1u << lane) - 1u));
-        if (sel && pos < count) out[pos] = j;
-        base += __popc(smask);
-        tie_base += __popc(tmask);
-      }
-    }
-    if (lane == 0) counts[(size_t)bh * nT + row] = count;
+    select_row<MAXV>(S + (size_t)lr * nT, nT, top_p, k_min, counts + (size_t)bh * nT + row,
+                     idx + ((size_t)bh * nT + row) * (size_t)cap);
   }
 }
 
@@ -383,38 +490,51 @@ cudaError_t launch_rope_table(const Geom& g, int dt, int dh, int dw, float base,
   return cudaGetLastError();
 }
 
-size_t select_smem_bytes(int nT, int d, int rpw) {
-  const int R = 8 * rpw;
+size_t select_smem_bytes(int nT, int d, int R) {
   return sizeof(float) * ((size_t)d * R + (size_t)d * kKCS + (size_t)R * nT);
 }
 
-template <int RPW, int D>
-static cudaError_t launch_select_t(const Geom& g, const float* qp, const float* kp, float top_p, int k_min,
+// Rows per block: the largest of 32, 16, 8, 4 whose score block fits.
+int select_rows(int nT, int d) {
+  for (int R = 32; R > 4; R >>= 1)
+    if (select_smem_bytes(nT, d, R) <= 220 * 1024) return R;
+  return 4;
+}
+
+template <int D, int MAXV, int WARPS>
+static cudaError_t launch_select_v(const Geom& g, const float* qp, const float* kp, float top_p, int k_min,
                                    int* counts, int* idx, int cap, cudaStream_t s) {
-  const size_t smem = select_smem_bytes(g.nT, D, RPW);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<RPW, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int R = select_rows(g.nT, D);
+  if (R > 2 * WARPS) R = 2 * WARPS;
+  const size_t smem = select_smem_bytes(g.nT, D, R);
+  auto kern = select_kernel<D, MAXV, WARPS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  constexpr int R = 8 * RPW;
   dim3 grid((g.nT + R - 1) / R, g.BH);
-  select_kernel<RPW, D><<<grid, 256, smem, s>>>(g, qp, kp, top_p, k_min, counts, idx, cap);
+  kern<<<grid, WARPS * 32, smem, s>>>(g, qp, kp, top_p, k_min, counts, idx, cap, R);
   return cudaGetLastError();
 }
 
-// Rows per warp: 4 while the score block fits comfortably, else 1.
-int select_rows_per_warp(int nT, int d) { return select_smem_bytes(nT, d, 4) <= 220 * 1024 ? 4 : 1; }
+// Values per lane: the smallest supported multiple covering nT / 32.
+template <int D>
+static cudaError_t launch_select_t(const Geom& g, const float* qp, const float* kp, float top_p, int k_min,
+                                   int* counts, int* idx, int cap, cudaStream_t s) {
+  const int need = (g.nT + 31) / 32;
+  if (need <= 2) return launch_select_v<D, 2, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 4) return launch_select_v<D, 4, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 8) return launch_select_v<D, 8, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 16) return launch_select_v<D, 16, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 24) return launch_select_v<D, 24, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 40) return launch_select_v<D, 40, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (need <= 64) return launch_select_v<D, 64, 8>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  return launch_select_v<D, 128, 8>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+}
 
 cudaError_t launch_select(const Geom& g, const float* qp, const float* kp, float top_p, int k_min, int* counts,
                           int* idx, int cap, cudaStream_t s) {
-  const int rpw = select_rows_per_warp(g.nT, g.d);
-  if (g.d == 128)
-    return rpw == 4 ? launch_select_t<4, 128>(g, qp, kp, top_p, k_min, counts, idx, cap, s)
-                    : launch_select_t<1, 128>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (g.d == 64)
-    return rpw == 4 ? launch_select_t<4, 64>(g, qp, kp, top_p, k_min, counts, idx, cap, s)
-                    : launch_select_t<1, 64>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (g.d == 32)
-    return rpw == 4 ? launch_select_t<4, 32>(g, qp, kp, top_p, k_min, counts, idx, cap, s)
-                    : launch_select_t<1, 32>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (g.d == 128) return launch_select_t<128>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (g.d == 64) return launch_select_t<64>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
+  if (g.d == 32) return launch_select_t<32>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
   return cudaErrorInvalidValue;
 }
 

@@ -279,9 +279,11 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
               const float p1 = ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, -m_use));
               const float p2 = ex2(fmaf(__uint_as_float(s1[2 * c]), sl2, -m_use));
               const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, -m_use));
-              sum += (p0 + p1) + (p2 + p3);
               pk[c] = pack_bf16(p0, p1);
               pk[16 + c] = pack_bf16(p2, p3);
+              // normalise with the probabilities as the MMA sees them (bf16)
+              sum += (__uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u)) +
+                     (__uint_as_float(pk[16 + c] << 16) + __uint_as_float(pk[16 + c] & 0xFFFF0000u));
             }
             l += sum;
           } else {

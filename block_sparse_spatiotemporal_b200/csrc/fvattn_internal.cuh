@@ -50,6 +50,7 @@ struct WsLayout {
   size_t counts, idx;    // int32 [BH*nT], [BH*nT*nT] (forward without cache)
   size_t uni, ucount;    // int32 [BH*P*nT], [BH*P]
   size_t worklist;       // int32 [BH*P]
+  size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
   size_t total;
 };
@@ -285,7 +286,7 @@ cudaError_t launch_select(const Geom& g, const float* qp, const float* kp, float
                           int* idx, int cap, cudaStream_t s);
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
                          cudaStream_t s);
-cudaError_t launch_rank(const int* key, int n, int* worklist, cudaStream_t s);
+cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s);
 cudaError_t launch_fine_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineTcArgs& a,
                            int num_sms, cudaStream_t s);
 cudaError_t launch_fine_f32(const FineF32Args& a, cudaStream_t s);

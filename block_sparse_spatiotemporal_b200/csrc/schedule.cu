@@ -72,23 +72,31 @@ __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restric
 }
 
 // rank(e) = #{e' : key(e') > key(e)} + #{e' < e : key(e') == key(e)};
-// worklist[rank(e)] = e.  Keys staged through shared memory in chunks.
-__global__ void __launch_bounds__(256) rank_kernel(const int* __restrict__ key, int n, int* __restrict__ worklist) {
-  __shared__ int ks[2048];
+// worklist[rank(e)] = e.  The comparisons are split over segments of e'
+// (grid y) whose partial counts are added into rank[] (integer adds, so the
+// result does not depend on their order); a second kernel scatters.
+constexpr int kRankSeg = 1024;
+
+__global__ void __launch_bounds__(256) rank_partial_kernel(const int* __restrict__ key, int n, int* __restrict__ rank) {
+  __shared__ int ks[kRankSeg];
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  const int ke = e < n ? key[e] : 0;
-  int rank = 0;
-  for (int c0 = 0; c0 < n; c0 += 2048) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < 2048 && c0 + i < n; i += blockDim.x) ks[i] = key[c0 + i];
-    __syncthreads();
-    const int lim = min(2048, n - c0);
-    for (int i = 0; i < lim; ++i) {
-      const int kk = ks[i];
-      rank += (kk > ke || (kk == ke && c0 + i < e)) ? 1 : 0;
-    }
+  const int s0 = blockIdx.y * kRankSeg;
+  const int len = min(kRankSeg, n - s0);
+  for (int i = threadIdx.x; i < len; i += blockDim.x) ks[i] = key[s0 + i];
+  __syncthreads();
+  if (e >= n) return;
+  const int ke = key[e];
+  int c = 0;
+  for (int i = 0; i < len; ++i) {
+    const int kk = ks[i];
+    c += (kk > ke || (kk == ke && s0 + i < e)) ? 1 : 0;
   }
-  if (e < n) worklist[rank] = e;
+  if (c) atomicAdd(&rank[e], c);
+}
+
+__global__ void scatter_rank_kernel(const int* __restrict__ rank, int n, int* __restrict__ worklist) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < n) worklist[rank[e]] = e;
 }
 
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
@@ -100,8 +108,12 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
   return cudaGetLastError();
 }
 
-cudaError_t launch_rank(const int* key, int n, int* worklist, cudaStream_t s) {
-  rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(key, n, worklist);
+cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(rank, 0, sizeof(int) * (size_t)n, s);
+  if (e != cudaSuccess) return e;
+  dim3 grid((n + 255) / 256, (n + kRankSeg - 1) / kRankSeg);
+  rank_partial_kernel<<<grid, 256, 0, s>>>(key, n, rank);
+  scatter_rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(rank, n, worklist);
   return cudaGetLastError();
 }
 

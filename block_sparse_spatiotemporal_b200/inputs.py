@@ -9,9 +9,10 @@ The pages measure on real Wan / Mochi activations ("FVAttn" page, section 03;
 "CalibAtt" page, "Demonstrated performance"), which are not available here.
 These tensors stand in for them.
 
-Recipe (fixed draw order, numpy ``default_rng(seed)``):
+Recipe (numpy generators; every stream is seeded, so the tensors do not
+depend on the number of threads that draw them):
 
-1. For each head h in order:
+1. Head parameters, from ``default_rng(seed)`` in this order, head by head:
    a. concentration s_h and bandwidth sigma_h: fixed (s=3, sigma=0.15) for
       the "fixed" generator, else s_h = exp(U[log 1, log 6]) then
       sigma_h = U[0.05, 0.3];
@@ -19,8 +20,9 @@ Recipe (fixed draw order, numpy ``default_rng(seed)``):
    c. phases b_h, shape [D], drawn U[0, 2*pi);
    d. with sinks: 2 distinct sink tiles, ``choice(nT, 2, replace=False)``
       over raster-cube tile ids.
-2. Noise, in this order: Q noise for heads 0..H-1, then K noise for heads
-   0..H-1, then V for heads 0..H-1, each [N, d] standard normal (float32).
+2. Noise: tensor t (0 = Q noise, 1 = K noise, 2 = V) of head h of batch b is
+   [N, d] standard normal (float32) from
+   ``default_rng(SeedSequence([seed, 1 + t, b, h]))``.
 3. phi(x)_j = cos(omega_j . x + b_j) with x = (t, h, w) / max(extent - 1, 1)
    the normalised coordinate of the token (unnormalised features, so that
    logits are large and attention is spatially local).
@@ -30,8 +32,10 @@ Recipe (fixed draw order, numpy ``default_rng(seed)``):
    stay float32.
 
 Perturbed steps for the cached-mask mode: Q_t = Q_{t-1} + 0.05 * N(0,1) and
-K_t likewise (cumulative over t, float32 masters, drawn Q then K per step,
-heads in order), V fixed; each step is rounded to bf16 on its own.
+K_t likewise (cumulative over t, float32 masters), V fixed; the noise of
+step t, tensor t' (0 = Q, 1 = K), head h comes from
+``default_rng(SeedSequence([seed, 100 + t, t', b, h]))``; each step is
+rounded to bf16 on its own.
 
 Token layout: natural order is raster order over the latent grid (T, Hg, W),
 index n = (t * Hg + h) * W + w, tensors are [B, H, N, d] with B = 1.
@@ -156,13 +160,24 @@ def _finish(x32, wl):
     return f32_to_bf16_bits(x32) if wl.dtype == "bf16" else x32.astype(np.float32)
 
 
+def _noise(seed_words, shape):
+    return np.random.default_rng(np.random.SeedSequence(seed_words)).standard_normal(shape, dtype=np.float32)
+
+
+def _parallel(fn, items):
+    import concurrent.futures
+    import os
+    workers = max(1, min(len(items), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        list(ex.map(fn, items))
+
+
 def make_inputs(wl: Workload, keep_f32_masters: bool = False):
     """Draw (q, k, v) for a workload, shapes [B, H, N, d].
 
     bf16 workloads return uint16 arrays of bf16 bit patterns, fp32 workloads
     float32 arrays.  With ``keep_f32_masters`` the float32 Q/K before rounding
-    and the generator state are returned too (for the perturbed steps).
-    """
+    are returned too (for the perturbed steps)."""
     rng = np.random.default_rng(wl.seed)
     params = _head_params(rng, wl)
     T, Hg, W = wl.grid
@@ -176,43 +191,39 @@ def make_inputs(wl: Workload, keep_f32_masters: bool = False):
     v = np.empty((B, H, N, d), out_dtype)
     qm = np.empty((B, H, N, d), np.float32) if keep_f32_masters else None
     km = np.empty((B, H, N, d), np.float32) if keep_f32_masters else None
+    sink_rows = [None if p[4] is None else _sink_rows(wl, p[4]) for p in params]
 
-    def phi(h):
+    def one(bh):
+        b, h = bh
         s, _, omega, phase, _ = params[h]
-        return (s * np.cos(x @ omega.T + phase)).astype(np.float32)
+        phi = (s * np.cos(x @ omega.T + phase)).astype(np.float32)
+        qh = phi + np.float32(0.3) * _noise([wl.seed, 1, b, h], (N, d))
+        kh = phi + np.float32(0.3) * _noise([wl.seed, 2, b, h], (N, d))
+        if sink_rows[h] is not None:
+            kh[sink_rows[h]] *= np.float32(3.0)
+        if keep_f32_masters:
+            qm[b, h] = qh
+            km[b, h] = kh
+        q[b, h] = _finish(qh, wl)
+        k[b, h] = _finish(kh, wl)
+        v[b, h] = _finish(_noise([wl.seed, 3, b, h], (N, d)), wl)
 
-    for b in range(B):
-        for h in range(H):
-            qh = phi(h) + np.float32(0.3) * rng.standard_normal((N, d), dtype=np.float32)
-            if keep_f32_masters:
-                qm[b, h] = qh
-            q[b, h] = _finish(qh, wl)
-        for h in range(H):
-            kh = phi(h) + np.float32(0.3) * rng.standard_normal((N, d), dtype=np.float32)
-            sinks = params[h][4]
-            if sinks is not None:
-                kh[_sink_rows(wl, sinks)] *= np.float32(3.0)
-            if keep_f32_masters:
-                km[b, h] = kh
-            k[b, h] = _finish(kh, wl)
-        for h in range(H):
-            v[b, h] = _finish(rng.standard_normal((N, d), dtype=np.float32), wl)
+    _parallel(one, [(b, h) for b in range(B) for h in range(H)])
     if keep_f32_masters:
-        return q, k, v, dict(q_f32=qm, k_f32=km, rng=rng, params=params)
+        return q, k, v, dict(q_f32=qm, k_f32=km)
     return q, k, v
 
 
 def perturb_steps(wl: Workload, masters: dict, steps: int = 10):
     """Yield (q_t, k_t) for t = 1..steps: cumulative 0.05*N(0,1) perturbation
     of the float32 masters returned by ``make_inputs(..., keep_f32_masters=True)``."""
-    rng = masters["rng"]
     qm = masters["q_f32"].copy()
     km = masters["k_f32"].copy()
     B, H, N, d = qm.shape
-    for _ in range(steps):
-        for b in range(B):
-            for h in range(H):
-                qm[b, h] += np.float32(0.05) * rng.standard_normal((N, d), dtype=np.float32)
-            for h in range(H):
-                km[b, h] += np.float32(0.05) * rng.standard_normal((N, d), dtype=np.float32)
+    for t in range(1, steps + 1):
+        def one(bh, t=t):
+            b, h = bh
+            qm[b, h] += np.float32(0.05) * _noise([wl.seed, 100 + t, 0, b, h], (N, d))
+            km[b, h] += np.float32(0.05) * _noise([wl.seed, 100 + t, 1, b, h], (N, d))
+        _parallel(one, [(b, h) for b in range(B) for h in range(H)])
         yield _finish(qm, wl), _finish(km, wl)

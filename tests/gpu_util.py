@@ -51,13 +51,17 @@ def oracle_coarse(wl: Workload, q, k, top_p, k_min, b=0, heads=None):
 def compare_blocks(res: dict, gpu_counts: np.ndarray, gpu_idx: np.ndarray, top_p: float):
     """Compare one head's GPU lists with the oracle's.
 
-    Returns (n_mismatch, n_border, n_neartie_checked, equal_rows): rows whose
-    cumulative mass is within 1e-5 of top_p at the cut are exempt (counted);
-    near-tie rows whose GPU set differs must still be a valid top-count set;
-    any other difference is a mismatch."""
-    P, counts, idx, border = res["P"], res["counts"], res["idx"], res["border"]
-    nT = P.shape[0]
-    near = O.near_tie_rows(P, counts)
+    Returns (n_mismatch, n_border, n_neartie_checked, equal_rows).  Rows whose
+    cumulative mass lies within 1e-5 of top_p at the cut are exempt (counted).
+    Near-tie rows -- the last kept and first dropped logits closer than the
+    float32 rounding bound of a 128-term dot product (1e-5 of the row's
+    largest scale * |Qp|.|Kp|) -- may select either tile, but the GPU set must
+    still be a top-count set within that bound.  Any other difference is a
+    mismatch."""
+    S, counts, idx, border = res["S"], res["counts"], res["idx"], res["border"]
+    nT = S.shape[0]
+    tol = 1e-5 * res["s_abs"].max(axis=1)
+    near = O.near_tie_rows(S, counts, tol)
     mism = 0
     ntie = 0
     equal = np.zeros(nT, bool)
@@ -72,7 +76,7 @@ def compare_blocks(res: dict, gpu_counts: np.ndarray, gpu_idx: np.ndarray, top_p
             ok = len(set(sel.tolist())) == c and (np.diff(sel) > 0).all()
             rest = np.setdiff1d(np.arange(nT), sel)
             if ok and len(rest):
-                ok = P[r, sel].min() >= P[r, rest].max() * (1 - 1e-6)
+                ok = S[r, sel].min() >= S[r, rest].max() - tol[r]
             ntie += 1
             if ok:
                 continue
