@@ -61,7 +61,7 @@ int make_geom(const fvattn_shape* s, Geom* g) {
   g->nT = (int)nT;
   g->N = (int)N;
   g->BH = (int)BH;
-  g->P = (int)((nT + 1) / 2);
+  g->P = (int)((nT + kItemTiles - 1) / kItemTiles);
   g->order = s->order;
   g->scale = s->scale > 0.f ? s->scale : (float)(1.0 / std::sqrt((double)d));
   return FVATTN_OK;

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/fvattn.h"
+#include "fvattn.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "fvattn kernels are written for sm_100a (B200) only"
@@ -15,6 +15,7 @@
 namespace fvattn {
 
 constexpr int kTileTokens = 64;
+constexpr int kItemTiles = 4;   // query tiles per fine-stage work item (two 128-row streams)
 constexpr int kMaxTiles = 8192;
 
 // Device status codes (workspace status word).
@@ -34,7 +35,7 @@ struct Geom {
   int nT;                // tiles per head
   int N;                 // tokens per head
   int BH;
-  int P;                 // query-tile pairs per head = ceil(nT/2)
+  int P;                 // fine-stage work items per head = ceil(nT / kItemTiles)
   int order;             // fvattn_order
   float scale;           // softmax scale
 };
@@ -138,6 +139,20 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of the phase with the given parity (for polling loops;
+// try_wait may suspend the thread for a while before it reports failure).
+__device__ inline bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)

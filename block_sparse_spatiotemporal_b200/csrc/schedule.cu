@@ -2,36 +2,41 @@
 // runtime head-level load balancing (section 02), applied across the SMs of
 // one GPU instead of across GPUs.
 //
-// A work item is a pair of adjacent query tiles (2p, 2p+1) of one (batch,
-// head): the pair fills the 128 rows of one tensor-core tile, and the item
-// walks the union of the two tiles' key lists, each entry tagged with which
-// tile selected it (the other tile's rows are masked for that key tile).
-// Items are then ranked by union size, longest first (LPT), ties by item
-// code, so the persistent fine kernel hands the heavy items out first and
-// the light ones fill the tail.
+// A work item is four adjacent query tiles 4q .. 4q+3 of one (batch, head):
+// two 128-row tensor-core streams, A = tiles (4q, 4q+1) and B = tiles
+// (4q+2, 4q+3), that share every K/V tile the item loads.  The item walks
+// the union of the four tiles' key lists; each entry records which of the
+// four tiles selected it (the other tiles' rows are masked for it), which
+// stream takes part in it, and each stream's last entry.  Items are ranked by
+// union size, longest first (LPT), ties by item code, so the persistent fine
+// kernel hands the heavy items out first and the light ones fill the tail.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
 
-// One warp per item.  Entries: tile | (mask << 16), mask bit 0 = tile 2p
-// selected it, bit 1 = tile 2p+1.  Ascending tile ids.  Validates the lists:
-// counts in [0, nT], ids in [0, nT) and strictly ascending; violations set
-// kStatusBadBlock and the offending entries are dropped.
+// Entry word of the union list.
+//   bits  0-15  key tile id
+//   bits 16-19  selected by tile 4q+0 .. 4q+3
+//   bits 20-21  stream A / B takes part (a selecting tile, or the stream's
+//               one forced step when none of its tiles selected anything)
+//   bits 22-23  last entry of stream A / B in this item
+// One warp per item.  Validates the lists: counts in [0, nT], ids in
+// [0, nT) and strictly ascending; violations set kStatusBadBlock and the
+// offending entries are dropped.
 __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restrict__ counts,
                                                     const int* __restrict__ idx, int cap, int* __restrict__ uni,
                                                     int* __restrict__ ucount, int* status) {
-  extern __shared__ uint32_t bm[];  // per warp: 2 bitmaps of ceil(nT/32) words
+  extern __shared__ uint32_t bm[];  // per warp: 4 bitmaps of ceil(nT/32) words
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = (g.nT + 31) / 32;
-  uint32_t* bma = bm + warp * 2 * words;
-  uint32_t* bmb = bma + words;
+  uint32_t* bmw = bm + warp * 4 * words;
   const long long item = (long long)blockIdx.x * 4 + warp;
   if (item >= (long long)g.BH * g.P) return;
-  const int bh = (int)(item / g.P), p = (int)(item % g.P);
-  for (int w = lane; w < 2 * words; w += 32) bma[w] = 0u;
+  const int bh = (int)(item / g.P), qd = (int)(item % g.P);
+  for (int w = lane; w < 4 * words; w += 32) bmw[w] = 0u;
   __syncwarp();
-  for (int half = 0; half < 2; ++half) {
-    const int tile = 2 * p + half;
+  for (int t = 0; t < kItemTiles; ++t) {
+    const int tile = kItemTiles * qd + t;
     if (tile >= g.nT) break;
     const size_t row = (size_t)bh * g.nT + tile;
     int c = counts[row];
@@ -40,7 +45,7 @@ __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restric
       c = c < 0 ? 0 : g.nT;
     }
     const int* list = idx + row * (size_t)cap;
-    uint32_t* bmx = half ? bmb : bma;
+    uint32_t* bmx = bmw + t * words;
     for (int e = lane; e < c; e += 32) {
       const int j = list[e];
       const bool ok = j >= 0 && j < g.nT && (e == 0 || list[e - 1] < j);
@@ -53,20 +58,38 @@ __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restric
   }
   __syncwarp();
   int* out = uni + item * (long long)g.nT;
-  int n = 0;
+  int n = 0, lastA = -1, lastB = -1;
   for (int w = 0; w < words; ++w) {
     const int j = w * 32 + lane;
-    const uint32_t a = (bma[w] >> lane) & 1u, b = (bmb[w] >> lane) & 1u;
-    const uint32_t m = a | (b << 1);
-    const unsigned bal = __ballot_sync(0xffffffffu, m != 0u);
-    if (m) out[n + __popc(bal & ((1u << lane) - 1u))] = j | (int)(m << 16);
+    uint32_t sel = 0;
+#pragma unroll
+    for (int t = 0; t < kItemTiles; ++t) sel |= ((bmw[t * words + w] >> lane) & 1u) << t;
+    const uint32_t part = ((sel & 3u) ? 1u : 0u) | ((sel & 12u) ? 2u : 0u);
+    const unsigned bal = __ballot_sync(0xffffffffu, sel != 0u);
+    const int pos = n + __popc(bal & ((1u << lane) - 1u));
+    if (sel) out[pos] = j | (int)(sel << 16) | (int)(part << 20);
+    const unsigned ba = __ballot_sync(0xffffffffu, (part & 1u) != 0u);
+    const unsigned bb = __ballot_sync(0xffffffffu, (part & 2u) != 0u);
+    if (ba) lastA = n + __popc(bal & ((2u << (31 - __clz(ba))) - 1u)) - 1;
+    if (bb) lastB = n + __popc(bal & ((2u << (31 - __clz(bb))) - 1u)) - 1;
     n += __popc(bal);
   }
+  __syncwarp();
   if (lane == 0) {
-    if (n == 0) {  // both rows empty: one fully masked step keeps the item well formed
+    if (n == 0) {  // no tile selected anything: one step, fully masked, for both streams
       out[0] = 0;
       n = 1;
     }
+    if (lastA < 0) {  // stream A without a selection: it takes part in entry 0, masked
+      out[0] |= 1 << 20;
+      lastA = 0;
+    }
+    if (lastB < 0) {
+      out[0] |= 1 << 21;
+      lastB = 0;
+    }
+    out[lastA] |= 1 << 22;
+    out[lastB] |= 1 << 23;
     ucount[item] = n;
   }
 }
@@ -103,7 +126,7 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
                          cudaStream_t s) {
   const long long items = (long long)g.BH * g.P;
   const int words = (g.nT + 31) / 32;
-  const size_t smem = (size_t)4 * 2 * words * sizeof(uint32_t);
+  const size_t smem = (size_t)4 * 4 * words * sizeof(uint32_t);
   union_kernel<<<(unsigned)((items + 3) / 4), 128, smem, s>>>(g, counts, idx, cap, uni, ucount, status);
   return cudaGetLastError();
 }

@@ -155,12 +155,12 @@ int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void* q, const v
                                const fvattn_blocks* out, fvattn_stream_t stream);
 
 /* Schedule of the fine stage (single-GPU analogue of the "FVAttn" digest's
- * runtime head-level load balancing, section 02): work items are pairs of
- * adjacent query tiles (2p, 2p+1) of one (batch, head), encoded
- * ((b*H + h)*P + p) with P = ceil(nT/2); the cost of an item is the size of
- * the union of the two tiles' lists (the single tile's list for the last
- * item of an odd nT); items are sorted by cost descending, ties by ascending
- * item code (longest-processing-time first).  worklist has B*H*P int32. */
+ * runtime head-level load balancing, section 02): a work item is four
+ * adjacent query tiles 4q .. 4q+3 of one (batch, head), encoded
+ * ((b*H + h)*P + q) with P = ceil(nT/4); its cost is the size of the union
+ * of the four tiles' lists (tiles past nT contribute nothing); items are
+ * sorted by cost descending, ties by ascending item code
+ * (longest-processing-time first).  worklist has B*H*P int32. */
 int fvattn_build_worklist(const fvattn_shape* shape, const fvattn_blocks* blocks,
                           int32_t* worklist, void* ws, size_t ws_bytes, fvattn_stream_t stream);
 

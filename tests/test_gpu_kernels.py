@@ -193,7 +193,12 @@ def test_empty_rows_and_bad_block_ids():
 
 
 def test_worklist_is_longest_union_first():
-    wl = small((8, 16, 16), heads=4)
+    wl = small((8, 8, 20), heads=4)         # nT = 20 tiles: 5 items per head
+    _worklist_case(wl)
+    _worklist_case(small((4, 8, 20), heads=3))   # nT = 10: the last item has 2 tiles
+
+
+def _worklist_case(wl):
     q, k, v, res, gc, gi = _pool_select_case(wl)
     shape = shape_of(wl)
     ws = F.workspace(shape)
@@ -202,13 +207,14 @@ def test_worklist_is_longest_union_first():
     oi = np.stack([r["idx"] for r in res])[None].astype(np.int32)
     cd, idd = torch.from_numpy(oc).cuda(), torch.from_numpy(oi).cuda()
     got = F.build_worklist(shape, cd, idd, ws).cpu().numpy()
-    P = (nT + 1) // 2
+    P = (nT + 3) // 4
     cost = []
     for h, r in enumerate(res):
         for p in range(P):
-            a = set(r["idx"][2 * p, :r["counts"][2 * p]].tolist())
-            b = set(r["idx"][2 * p + 1, :r["counts"][2 * p + 1]].tolist()) if 2 * p + 1 < nT else set()
-            cost.append(len(a | b))
+            u = set()
+            for t in range(4 * p, min(4 * p + 4, nT)):
+                u |= set(r["idx"][t, :r["counts"][t]].tolist())
+            cost.append(len(u))
     cost = np.array(cost)
     want = np.lexsort((np.arange(len(cost)), -cost))
     assert np.array_equal(got, want)
