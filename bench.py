@@ -344,7 +344,7 @@ def run_gpu(args, wl):
             "roofline": {"kernel": "fine_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{pk_kind} bf16 burst"},
-            "gpu_launches": sum(n for _, n in stages.values()) + args.steps * (1 if rope is None else 2),
+            "gpu_launches": sum(n for _, n in stages.values()),
             "clocks": clocks,
             "e2e": e2e,
         }

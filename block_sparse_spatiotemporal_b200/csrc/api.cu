@@ -92,8 +92,12 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r) {
   const size_t rope_pairs =
       rope_on(r) ? (size_t)g.T * (r->dt / 2) + (size_t)g.Hg * (r->dh / 2) + (size_t)g.W * (r->dw / 2) : 0;
   L.rope_tab = take(sizeof(float2) * rope_pairs);
-  L.qp = take(sizeof(float) * (size_t)g.BH * g.nT * g.d);
-  L.kp = take(sizeof(float) * (size_t)g.BH * g.nT * g.d);
+  const size_t pooled = sizeof(float) * (size_t)g.BH * g.nT * g.d;
+  L.qh = take(pooled);
+  L.ql = take(pooled);
+  L.kh = take(pooled);
+  L.kl = take(pooled);
+  L.scores = take(sizeof(float) * (size_t)g.BH * g.nT * g.nT);
   L.counts = take(sizeof(int) * (size_t)g.BH * g.nT);
   L.idx = take(sizeof(int) * (size_t)g.BH * g.nT * g.nT);
   L.uni = take(sizeof(int) * (size_t)g.BH * g.P * g.nT);
@@ -175,13 +179,30 @@ int make_tile_map(CUtensorMap* map, const void* base, const Geom& g, bool natura
   return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
+// TMA descriptor over a pooled fp32 [BH, nT, d] tensor (tf32 operand of the
+// score kernel): 3D (d, nT, BH), box = 32 dims (128 bytes) x 128 tiles,
+// 128-byte swizzle; tiles past nT read as zero.
+int make_pooled_map(CUtensorMap* map, const float* base, const Geom& g) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FVATTN_ERR_CUDA;
+  const cuuint64_t row = (cuuint64_t)g.d * 4;
+  const cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.nT, (cuuint64_t)g.BH};
+  const cuuint64_t strides[2] = {row, row * (cuuint64_t)g.nT};
+  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Optional per-stage timing with CUDA events (host objects only).
 // ---------------------------------------------------------------------------
 struct Profiler {
   std::mutex mu;
   bool on = false;
-  struct Rec { int stage; cudaEvent_t a, b; };
+  struct Rec { int stage; cudaEvent_t a, b; int kernels; };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
 
@@ -204,6 +225,7 @@ Profiler& prof() {
 // Records events around one launch when profiling is on.
 struct StageTimer {
   int stage;
+  int kernels = 0;       // kernels this stage launched (for the launch count)
   cudaStream_t s;
   cudaEvent_t a = nullptr, b = nullptr;
   StageTimer(int st, cudaStream_t stream) : stage(st), s(stream) {
@@ -219,7 +241,7 @@ struct StageTimer {
     cudaEventRecord(b, s);
     Profiler& p = prof();
     std::lock_guard<std::mutex> lock(p.mu);
-    p.recs.push_back({stage, a, b});
+    p.recs.push_back({stage, a, b, kernels});
   }
 };
 
@@ -258,6 +280,7 @@ int begin(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws,
 int tables(const Call& c, const fvattn_rope* rope, bool need_tok) {
   StageTimer t(FVATTN_STAGE_TABLES, c.s);
   FV_CUDA(launch_tile_table(c.g, c.at<int>(c.L.tile_cube), c.at<int>(c.L.cube_rank), c.s));
+  t.kernels = 1 + (need_tok ? 1 : 0) + (rope_on(rope) ? 1 : 0);
   if (need_tok) FV_CUDA(launch_tile_token(c.g, c.at<int>(c.L.cube_rank), c.at<int>(c.L.tile_tok), c.s));
   if (rope_on(rope))
     FV_CUDA(launch_rope_table(c.g, rope->dt, rope->dh, rope->dw, rope->base, c.at<float2>(c.L.rope_tab), c.s));
@@ -275,17 +298,31 @@ int check_blocks(const fvattn_blocks* b, const Geom& g) {
 int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
                bool natural, bool pooled, bool rot, float top_p, int k_min, const fvattn_blocks* blocks) {
   const bool r = rope_on(rope);
+  PooledOut po{};
+  if (pooled) {
+    po.hi[0] = c.at<float>(c.L.qh);
+    po.lo[0] = c.at<float>(c.L.ql);
+    po.hi[1] = c.at<float>(c.L.kh);
+    po.lo[1] = c.at<float>(c.L.kl);
+  }
   {
   StageTimer t(FVATTN_STAGE_POOL, c.s);
   FV_CUDA(launch_pool(c.g, shape->dtype, q, k, natural ? 1 : 0, c.at<int>(c.L.tile_cube), c.at<int>(c.L.tile_tok),
                       r ? 1 : 0, r ? rope->dt : 0, r ? rope->dh : 0, r ? rope->dw : 0, c.at<float2>(c.L.rope_tab),
-                      pooled ? c.at<float>(c.L.qp) : nullptr, pooled ? c.at<float>(c.L.kp) : nullptr,
-                      rot ? c.at<void>(c.L.qrot) : nullptr, rot ? c.at<void>(c.L.krot) : nullptr, c.s));
+                      po, rot ? c.at<void>(c.L.qrot) : nullptr, rot ? c.at<void>(c.L.krot) : nullptr, c.s));
+  t.kernels = 1;
   }
+  if (!pooled) return FVATTN_OK;
   StageTimer t(FVATTN_STAGE_SELECT, c.s);
-  if (pooled)
-    FV_CUDA(launch_select(c.g, c.at<float>(c.L.qp), c.at<float>(c.L.kp), top_p, k_min, blocks->counts, blocks->idx,
-                          blocks->cap, c.s));
+  CUtensorMap mqh, mql, mkh, mkl;
+  FV_TRY(make_pooled_map(&mqh, po.hi[0], c.g));
+  FV_TRY(make_pooled_map(&mql, po.lo[0], c.g));
+  FV_TRY(make_pooled_map(&mkh, po.hi[1], c.g));
+  FV_TRY(make_pooled_map(&mkl, po.lo[1], c.g));
+  ScoreArgs sa{c.g, c.at<float>(c.L.scores), c.status, kDefaultWaitCap};
+  FV_CUDA(launch_scores(mqh, mql, mkh, mkl, sa, c.s));
+  FV_CUDA(launch_select(c.g, sa.S, top_p, k_min, blocks->counts, blocks->idx, blocks->cap, c.s));
+  t.kernels = 2;
   return FVATTN_OK;
 }
 
@@ -294,6 +331,7 @@ int run_schedule(const Call& c, const fvattn_blocks* blocks, int* worklist) {
   FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
                        c.status, c.s));
   FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, c.at<int>(c.L.rank), worklist, c.s));
+  t.kernels = 3;      // union, partial ranks, scatter
   return FVATTN_OK;
 }
 
@@ -326,6 +364,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.wait_cap = kDefaultWaitCap;
     StageTimer t(FVATTN_STAGE_FINE, c.s);
     FV_CUDA(launch_fine_tc(mq, mk, mv, a, c.dev.sms, c.s));
+    t.kernels = a.n_items > 0 ? 1 : 0;
   } else {
     FineF32Args a{};
     a.g = c.g;
@@ -345,6 +384,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.status = c.status;
     StageTimer t(FVATTN_STAGE_FINE, c.s);
     FV_CUDA(launch_fine_f32(a, c.s));
+    t.kernels = 1;
   }
   return FVATTN_OK;
 }
@@ -387,6 +427,7 @@ int fvattn_tile_reorder(const fvattn_shape* shape, const void* x, void* y, int32
   FV_TRY(tables(c, nullptr, false));
   StageTimer t(FVATTN_STAGE_REORDER, c.s);
   FV_CUDA(launch_reorder(c.g, c.at<int>(c.L.cube_rank), x, y, row_bytes, inverse ? 1 : 0, c.dev.sms, c.s));
+  t.kernels = 1;
   return FVATTN_OK;
 }
 
@@ -506,7 +547,7 @@ int fvattn_profile_read(double* ms, int64_t* launches) {
     if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
       st = FVATTN_ERR_CUDA;
     acc[r.stage] += t;
-    cnt[r.stage] += 1;
+    cnt[r.stage] += r.kernels;
     p.pool.push_back(r.a);
     p.pool.push_back(r.b);
   }

@@ -1,5 +1,6 @@
-// Coarse stage: 3D RoPE on load, tile mean-pooling, pooled scores, row
-// softmax and top-p selection with a k_min floor.
+// Coarse stage: 3D RoPE on load, tile mean-pooling, row softmax of the
+// pooled scores and top-p selection with a k_min floor.  The pooled score
+// GEMM itself runs on the tensor cores (scores_tc.cu).
 //
 //   "VSA" digest, section 3: the coarse stage pools each (4,4,4) cube and
 //     predicts per-tile importance;
@@ -10,11 +11,9 @@
 // Selection rule (per query-tile row of the coarse softmax P): m is the
 // fewest tiles, at least one, whose probabilities summed in descending order
 // (ties to the lower tile id) reach top_p; count = min(nT, max(m, k_min));
-// top_p >= 1 keeps every tile.  The kernel never sorts the row: it finds the
-// cut by bisection over the bit patterns of e_j = exp(s_j - max) (a radix
-// select; positive floats order like their bits), with every mass computed
-// as a deterministic warp-tree sum, and compares masses against top_p * Z
-// instead of dividing.
+// top_p >= 1 keeps every tile.  The kernel never sorts the row (see
+// select_row), computes every mass as a deterministic warp-tree sum, and
+// compares masses against top_p * Z instead of dividing.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
@@ -122,19 +121,28 @@ __device__ inline void rope_pair(const RopeArgs& r, const Geom& g, int dim, int 
 // w, w+4, ..., each lane DPL consecutive dims of the row (a warp reads one
 // whole row per step).  Sums are fp32 in a fixed order: rows of a warp in
 // sequence, then the 4 warp partials in warp order; mean = sum / 64.
-// Optionally writes the rotated rows, rounded to T, at tiled positions.
+// The mean is stored as two tf32 values, hi = rn_tf32(mean) and
+// lo = rn_tf32(mean - hi) (the subtraction is exact), row-major [BH][nT][d],
+// the operands of the tensor-core score kernel.  Optionally writes the
+// rotated rows, rounded to T, at tiled positions.
 // --------------------------------------------------------------------------
+__device__ inline float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__ q, const T* __restrict__ k,
                                                    int natural, const int* __restrict__ tile_cube,
-                                                   const int* __restrict__ tile_tok, RopeArgs rope,
-                                                   float* __restrict__ qp, float* __restrict__ kp,
+                                                   const int* __restrict__ tile_tok, RopeArgs rope, PooledOut po,
                                                    T* __restrict__ qrot, T* __restrict__ krot) {
   constexpr int DPL = D / 32;
   __shared__ float part[4][D];
   const int j = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const T* x = which == 0 ? q : k;
-  float* pooled = which == 0 ? qp : kp;
+  float* hi = po.hi[which];
+  float* lo = po.lo[which];
   T* rot = which == 0 ? qrot : krot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cube = tile_cube[j];
@@ -161,20 +169,21 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
       Vec<T, DPL>::store(dst, v);
     }
   }
-  if (!pooled) return;
+  if (!hi) return;
 #pragma unroll
   for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = acc[i];
   __syncthreads();
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    const float s = ((part[0][c] + part[1][c]) + part[2][c]) + part[3][c];
-    pooled[((size_t)bh * g.nT + j) * D + c] = s * (1.0f / 64.0f);
+    const float mean = (((part[0][c] + part[1][c]) + part[2][c]) + part[3][c]) * (1.0f / 64.0f);
+    const float h = round_tf32(mean);
+    const size_t at = ((size_t)bh * g.nT + j) * D + c;
+    hi[at] = h;
+    lo[at] = round_tf32(mean - h);
   }
 }
 
 // --------------------------------------------------------------------------
-// Score + select.  Block = 16 warps handling R <= 32 consecutive query tiles
-// of one head.  Phase 1 computes S[R][nT] = scale * Qp Kp^T (fp32 FFMA) into
-// shared memory.  Phase 2: warp w selects rows w and w + 16.
+// Selection, one warp per query-tile row of S = scale * Qp Kp^T.
 //
 // Tiles are ranked by their logit (the probability order; exp(s - max)
 // underflows to 0 for distant tiles, the logit does not), descending, ties
@@ -208,32 +217,34 @@ __device__ inline uint32_t order_key(float v) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-constexpr int kKC = 64;          // key tiles per phase-1 chunk
-constexpr int kKCS = 66;         // padded chunk row stride (floats)
+constexpr int kSelWarps = 8;     // rows (warps) per selection block
 constexpr int kMaxRounds = 32;   // argmax rounds before falling back to bisection
 
-// Selection of one row; srow holds the row's nT logits on entry and the
-// probabilities' numerators e_j = exp(s_j - max) on exit.
+// Selection of one row: src holds the row's nT logits; the probabilities'
+// numerators e_j = exp(s_j - max) go to the warp's shared scratch row srow.
 template <int MAXV>
-__device__ void select_row(float* srow, int nT, float top_p, int k_min, int* count_out, int* list) {
+__device__ void select_row(const float* __restrict__ src, float* srow, int nT, float top_p, int k_min,
+                           int* count_out, int* list) {
   constexpr int NW = (MAXV + 31) / 32;
   const int lane = threadIdx.x & 31;
   float v[MAXV];
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int j = i * 32 + lane;
-    v[i] = j < nT ? srow[j] : -INFINITY;
+    v[i] = j < nT ? __ldcs(src + j) : -INFINITY;
   }
   float mx = -INFINITY;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) mx = fmaxf(mx, v[i]);
   mx = warp_max(mx);
   float zp = 0.f;
+  const float mx2 = mx * 1.4426950408889634f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int j = i * 32 + lane;
     if (j < nT) {
-      const float e = expf(v[i] - mx);
+      float e;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fmaf(v[i], 1.4426950408889634f, -mx2)));
       srow[j] = e;
       zp += e;
     }
@@ -398,88 +409,39 @@ __device__ void select_row(float* srow, int nT, float top_p, int k_min, int* cou
   if (lane == 0) *count_out = count;
 }
 
-template <int D, int MAXV, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) select_kernel(Geom g, const float* __restrict__ qp,
-                                                            const float* __restrict__ kp, float top_p, int k_min,
-                                                            int* __restrict__ counts, int* __restrict__ idx, int cap,
-                                                            int R) {
+template <int MAXV>
+__global__ void __launch_bounds__(kSelWarps * 32, MAXV <= 24 ? 3 : (MAXV <= 40 ? 2 : 1)) select_rows_kernel(Geom g, const float* __restrict__ S,
+                                                                    float top_p, int k_min, int* __restrict__ counts,
+                                                                    int* __restrict__ idx, int cap, int stride) {
   extern __shared__ __align__(16) float sm[];
-  float* qs = sm;                       // [D][R]    transposed query rows
-  float* ks = qs + D * R;               // [D][kKCS] transposed key chunk
-  float* S = ks + D * kKCS;             // [R][nT]
-  const int nT = g.nT;
-  const int bh = blockIdx.y;
-  const int row0 = blockIdx.x * R;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* qph = qp + (size_t)bh * nT * D;
-  const float* kph = kp + (size_t)bh * nT * D;
-
-  for (int i = threadIdx.x; i < D * R; i += blockDim.x) {
-    const int r = i / D, c = i % D;
-    qs[c * R + r] = (row0 + r < nT) ? qph[(size_t)(row0 + r) * D + c] : 0.f;
-  }
-  const bool two = R > WARPS;                     // rows warp and warp + WARPS
-  for (int kc = 0; kc < nT; kc += kKC) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < D * kKC; i += blockDim.x) {
-      const int kk = i / D, c = i % D;
-      ks[c * kKCS + kk] = (kc + kk < nT) ? kph[(size_t)(kc + kk) * D + c] : 0.f;
-    }
-    __syncthreads();
-    if (warp < R) {
-      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        const float2 kv = *reinterpret_cast<const float2*>(&ks[c * kKCS + 2 * lane]);
-        const float q0 = qs[c * R + warp];
-        a00 = fmaf(q0, kv.x, a00);
-        a01 = fmaf(q0, kv.y, a01);
-        if (two) {
-          const float q1 = qs[c * R + warp + WARPS];
-          a10 = fmaf(q1, kv.x, a10);
-          a11 = fmaf(q1, kv.y, a11);
-        }
-      }
-      const int kk = kc + 2 * lane;
-      if (kk < nT) S[warp * nT + kk] = a00 * g.scale;
-      if (kk + 1 < nT) S[warp * nT + kk + 1] = a01 * g.scale;
-      if (two) {
-        if (kk < nT) S[(warp + WARPS) * nT + kk] = a10 * g.scale;
-        if (kk + 1 < nT) S[(warp + WARPS) * nT + kk + 1] = a11 * g.scale;
-      }
-    }
-  }
-  __syncthreads();
-
-  for (int lr = warp; lr < R; lr += WARPS) {
-    const int row = row0 + lr;
-    if (row >= nT) break;
-    select_row<MAXV>(S + (size_t)lr * nT, nT, top_p, k_min, counts + (size_t)bh * nT + row,
-                     idx + ((size_t)bh * nT + row) * (size_t)cap);
-  }
+  const int warp = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kSelWarps + warp;   // bh * nT + query tile
+  if (row >= (long long)g.BH * g.nT) return;
+  select_row<MAXV>(S + (size_t)row * g.nT, sm + (size_t)warp * stride, g.nT, top_p, k_min, counts + row,
+                   idx + (size_t)row * (size_t)cap);
 }
 
 template <typename T, int D>
 static cudaError_t launch_pool_t(const Geom& g, const void* q, const void* k, int natural, const int* tile_cube,
-                                 const int* tile_tok, const RopeArgs& rope, float* qp, float* kp, void* qrot,
+                                 const int* tile_tok, const RopeArgs& rope, const PooledOut& po, void* qrot,
                                  void* krot, cudaStream_t s) {
   dim3 grid(g.nT, g.BH, 2);
-  pool_kernel<T, D><<<grid, 128, 0, s>>>(g, (const T*)q, (const T*)k, natural, tile_cube, tile_tok, rope, qp, kp,
+  pool_kernel<T, D><<<grid, 128, 0, s>>>(g, (const T*)q, (const T*)k, natural, tile_cube, tile_tok, rope, po,
                                          (T*)qrot, (T*)krot);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pool(const Geom& g, int dtype, const void* q, const void* k, int natural, const int* tile_cube,
-                        const int* tile_tok, int rope_enabled, int dt, int dh, int dw, const float2* rope_tab, float* qp, float* kp,
-                        void* qrot, void* krot, cudaStream_t s) {
+                        const int* tile_tok, int rope_enabled, int dt, int dh, int dw, const float2* rope_tab,
+                        const PooledOut& po, void* qrot, void* krot, cudaStream_t s) {
   RopeArgs r{rope_enabled, dt, dh, dw, rope_tab};
   if (dtype == FVATTN_BF16) {
-    if (g.d == 128) return launch_pool_t<__nv_bfloat16, 128>(g, q, k, natural, tile_cube, tile_tok, r, qp, kp, qrot, krot, s);
-    if (g.d == 64) return launch_pool_t<__nv_bfloat16, 64>(g, q, k, natural, tile_cube, tile_tok, r, qp, kp, qrot, krot, s);
+    if (g.d == 128) return launch_pool_t<__nv_bfloat16, 128>(g, q, k, natural, tile_cube, tile_tok, r, po, qrot, krot, s);
+    if (g.d == 64) return launch_pool_t<__nv_bfloat16, 64>(g, q, k, natural, tile_cube, tile_tok, r, po, qrot, krot, s);
   } else {
-    if (g.d == 128) return launch_pool_t<float, 128>(g, q, k, natural, tile_cube, tile_tok, r, qp, kp, qrot, krot, s);
-    if (g.d == 64) return launch_pool_t<float, 64>(g, q, k, natural, tile_cube, tile_tok, r, qp, kp, qrot, krot, s);
-    if (g.d == 32) return launch_pool_t<float, 32>(g, q, k, natural, tile_cube, tile_tok, r, qp, kp, qrot, krot, s);
+    if (g.d == 128) return launch_pool_t<float, 128>(g, q, k, natural, tile_cube, tile_tok, r, po, qrot, krot, s);
+    if (g.d == 64) return launch_pool_t<float, 64>(g, q, k, natural, tile_cube, tile_tok, r, po, qrot, krot, s);
+    if (g.d == 32) return launch_pool_t<float, 32>(g, q, k, natural, tile_cube, tile_tok, r, po, qrot, krot, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -490,52 +452,35 @@ cudaError_t launch_rope_table(const Geom& g, int dt, int dh, int dw, float base,
   return cudaGetLastError();
 }
 
-size_t select_smem_bytes(int nT, int d, int R) {
-  return sizeof(float) * ((size_t)d * R + (size_t)d * kKCS + (size_t)R * nT);
-}
+// Shared scratch row stride: nT rounded up to 4 floats.
+static int select_stride(int nT) { return (nT + 3) & ~3; }
 
-// Rows per block: the largest of 32, 16, 8, 4 whose score block fits.
-int select_rows(int nT, int d) {
-  for (int R = 32; R > 4; R >>= 1)
-    if (select_smem_bytes(nT, d, R) <= 220 * 1024) return R;
-  return 4;
-}
-
-template <int D, int MAXV, int WARPS>
-static cudaError_t launch_select_v(const Geom& g, const float* qp, const float* kp, float top_p, int k_min,
-                                   int* counts, int* idx, int cap, cudaStream_t s) {
-  int R = select_rows(g.nT, D);
-  if (R > 2 * WARPS) R = 2 * WARPS;
-  const size_t smem = select_smem_bytes(g.nT, D, R);
-  auto kern = select_kernel<D, MAXV, WARPS>;
+template <int MAXV>
+static cudaError_t launch_select_v(const Geom& g, const float* S, float top_p, int k_min, int* counts, int* idx,
+                                   int cap, cudaStream_t s) {
+  const int stride = select_stride(g.nT);
+  const size_t smem = sizeof(float) * (size_t)kSelWarps * stride;
+  auto kern = select_rows_kernel<MAXV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((g.nT + R - 1) / R, g.BH);
-  kern<<<grid, WARPS * 32, smem, s>>>(g, qp, kp, top_p, k_min, counts, idx, cap, R);
+  const long long rows = (long long)g.BH * g.nT;
+  const unsigned blocks = (unsigned)((rows + kSelWarps - 1) / kSelWarps);
+  kern<<<blocks, kSelWarps * 32, smem, s>>>(g, S, top_p, k_min, counts, idx, cap, stride);
   return cudaGetLastError();
 }
 
 // Values per lane: the smallest supported multiple covering nT / 32.
-template <int D>
-static cudaError_t launch_select_t(const Geom& g, const float* qp, const float* kp, float top_p, int k_min,
-                                   int* counts, int* idx, int cap, cudaStream_t s) {
+cudaError_t launch_select(const Geom& g, const float* S, float top_p, int k_min, int* counts, int* idx, int cap,
+                          cudaStream_t s) {
   const int need = (g.nT + 31) / 32;
-  if (need <= 2) return launch_select_v<D, 2, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 4) return launch_select_v<D, 4, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 8) return launch_select_v<D, 8, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 16) return launch_select_v<D, 16, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 24) return launch_select_v<D, 24, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 40) return launch_select_v<D, 40, 16>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (need <= 64) return launch_select_v<D, 64, 8>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  return launch_select_v<D, 128, 8>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-}
-
-cudaError_t launch_select(const Geom& g, const float* qp, const float* kp, float top_p, int k_min, int* counts,
-                          int* idx, int cap, cudaStream_t s) {
-  if (g.d == 128) return launch_select_t<128>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (g.d == 64) return launch_select_t<64>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  if (g.d == 32) return launch_select_t<32>(g, qp, kp, top_p, k_min, counts, idx, cap, s);
-  return cudaErrorInvalidValue;
+  if (need <= 2) return launch_select_v<2>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 4) return launch_select_v<4>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 8) return launch_select_v<8>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 16) return launch_select_v<16>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 24) return launch_select_v<24>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 40) return launch_select_v<40>(g, S, top_p, k_min, counts, idx, cap, s);
+  if (need <= 64) return launch_select_v<64>(g, S, top_p, k_min, counts, idx, cap, s);
+  return launch_select_v<128>(g, S, top_p, k_min, counts, idx, cap, s);
 }
 
 }  // namespace fvattn

@@ -47,7 +47,9 @@ struct WsLayout {
   size_t cube_rank;      // int32 [nT]: tile rank of raster cube id
   size_t tile_tok;       // int32 [N]: natural token index of each tiled row
   size_t rope_tab;       // float2 [(T*dt + Hg*dh + W*dw)/2]: (cos, sin)
-  size_t qp, kp;         // float [BH*nT*d]
+  size_t qh, ql;         // float [BH*nT*d] pooled Q as tf32 hi + lo
+  size_t kh, kl;         // float [BH*nT*d] pooled K as tf32 hi + lo
+  size_t scores;         // float [BH*nT*nT] scaled coarse logits
   size_t counts, idx;    // int32 [BH*nT], [BH*nT*nT] (forward without cache)
   size_t uni, ucount;    // int32 [BH*P*nT], [BH*P]
   size_t worklist;       // int32 [BH*P]
@@ -60,6 +62,19 @@ struct WsLayout {
 struct RopeArgs {
   int enabled, dt, dh, dw;
   const float2* tab;     // [T*dt/2 | Hg*dh/2 | W*dw/2]
+};
+
+// Pooled means split into tf32 hi/lo parts; [0] = Q, [1] = K.
+struct PooledOut {
+  float* hi[2];
+  float* lo[2];
+};
+
+struct ScoreArgs {
+  Geom g;
+  float* S;              // [BH][nT][nT]
+  int* status;
+  long long wait_cap;
 };
 
 struct FineTcArgs {
@@ -174,6 +189,15 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* a
       return false;
     }
   }
+}
+
+// Wait that ignores `abort`: used on the way out to let copies or MMAs that
+// were already issued land before the block exits or frees TMEM.
+__device__ inline bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, long long cap) {
+  for (long long i = 0; i < cap; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  set_status(status, kStatusWaitCap);
+  return false;
 }
 
 __device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
@@ -296,9 +320,11 @@ cudaError_t launch_reorder(const Geom& g, const int* cube_rank, const void* x, v
 cudaError_t launch_rope_table(const Geom& g, int dt, int dh, int dw, float base, float2* tab, cudaStream_t s);
 cudaError_t launch_pool(const Geom& g, int dtype, const void* q, const void* k, int natural, const int* tile_cube,
                         const int* tile_tok, int rope_enabled, int dt, int dh, int dw, const float2* rope_tab,
-                        float* qp, float* kp, void* qrot, void* krot, cudaStream_t s);
-cudaError_t launch_select(const Geom& g, const float* qp, const float* kp, float top_p, int k_min, int* counts,
-                          int* idx, int cap, cudaStream_t s);
+                        const PooledOut& po, void* qrot, void* krot, cudaStream_t s);
+cudaError_t launch_scores(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                          const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s);
+cudaError_t launch_select(const Geom& g, const float* S, float top_p, int k_min, int* counts, int* idx, int cap,
+                          cudaStream_t s);
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
                          cudaStream_t s);
 cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s);

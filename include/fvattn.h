@@ -197,11 +197,11 @@ int fvattn_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t cap_iteratio
                                  fvattn_stream_t stream);
 
 /* Per-stage timing.  While enabled, every entry point records a pair of CUDA
- * events on its stream around each kernel it launches (host-side event
- * objects only; no device memory).  fvattn_profile_read synchronises on the
- * recorded events, writes the summed milliseconds and launch counts per
- * stage into ms[FVATTN_STAGE_COUNT] and launches[FVATTN_STAGE_COUNT]
- * (either may be NULL) and clears the record.  Not thread-safe against
+ * events on its stream around each stage it runs (host-side event objects
+ * only; no device memory).  fvattn_profile_read synchronises on the recorded
+ * events, writes per stage the summed milliseconds and the number of this
+ * library's kernels launched into ms[FVATTN_STAGE_COUNT] and
+ * launches[FVATTN_STAGE_COUNT] (either may be NULL) and clears the record.  Not thread-safe against
  * concurrent calls from several host threads. */
 typedef enum {
   FVATTN_STAGE_TABLES = 0,    /* tile / token / RoPE tables */
