@@ -2,93 +2,122 @@
 // token-level attention restricted to the selected tiles; "CalibAtt"
 // digest: selected connections computed densely, the rest skipped).
 //
-// Persistent kernel, one CTA per SM, 384 threads.  A work item is four
-// adjacent query tiles of one head, run as two 128-row streams that share
-// every K/V tile: stream A = tiles (4q, 4q+1), stream B = (4q+2, 4q+3).
-//   warp 0       TMA producer: the item's four Q tiles, then K/V of every
-//                entry of the item's union list into a 5-stage ring;
-//   warps 1, 2   MMA issuers, one thread per stream: for each entry the
-//                stream takes part in, S = Q K^T (M=128, N=64, K=128,
-//                operands in shared memory) into one of its two TMEM S
-//                buffers, then O += P V (M=128, N=128, K=64, P read from
-//                TMEM) of its previous step;
-//   warps 4-7    softmax of stream A, warps 8-11 softmax of stream B: thread
-//                r of a group owns row r (TMEM lane r) of its stream.
-// While one stream's softmax runs, the tensor core works on the other
-// stream.  A key tile selected by only some of an item's tiles is masked for
-// the others' rows: their P row is written as zeros and no exponential is
-// evaluated for them, so every row sees exactly its own tile's selection.
-// Online softmax in base 2 with a lazy rescale (O is rescaled in TMEM only
-// when a row's running max grows by more than 2^64); the normaliser sums the
-// bf16 probabilities the PV MMA consumes.
+// Persistent kernel, one CTA per SM, 384 threads.  A work item is two
+// adjacent query tiles of one head: one 128-row tensor-core tile walking the
+// union of the two tiles' key lists two entries (128 keys) per step.
+//   warp 0       TMA producer: the item's Q (double-buffered across items),
+//                K and V of every step's two key tiles into 2-stage rings
+//                (a load has about one softmax step of lead);
+//   warp 1       S issuer (one thread): S = Q K^T (M=128, N=128, K=128) of
+//                step c into TMEM S buffer c & 1 once the PV of step c - 2
+//                (the buffer's previous P) is complete;
+//   warp 2       PV issuer (one thread): O_t += P_t V_t (M=128, N=128,
+//                K=64) for the step's key tiles t = 0, 1 once P is written;
+//   warps 4-7    softmax of the first key tile of every step, warps 8-11 of
+//                the second: thread r of a group owns row r (TMEM lane r).
+// Each group keeps its own online-softmax state and its own O accumulator,
+// so the groups never synchronise per step; the epilogue merges the two
+// (m, l, O) triples.  A key tile selected by only one of the item's query
+// tiles is masked for the other tile's rows: their P row is written as zeros
+// and no exponential is evaluated for them, so every row sees exactly its
+// own tile's selection.  An item with an odd number of entries pads its last
+// step with a masked copy of its last key tile.
+// Online softmax in base 2 with a lazy rescale: a row keeps its reference
+// max m until a step's probabilities sum past 2^64, and only then is its O
+// rescaled in TMEM, so the max is evaluated once per item and on those rare
+// steps.  The normaliser sums the bf16 probabilities the PV MMA consumes.
+// The elementwise math runs on packed f32x2 instructions; exponentials can
+// be split between the MUFU unit and a polynomial on the FMA pipe (see
+// exp2_poly2).
 //
-// TMEM (512 columns), per stream s at column 256 s: S0 [0,64), S1 [64,128),
-// O [128,256), fp32; P (bf16) overwrites the first 32 columns of its S.
+// TMEM (512 columns): S buffers 0, 1 at [128 b, 128 b + 128), key tile t in
+// columns 64 t .. 64 t + 63 (its P, bf16, overwrites the first 32); O of
+// key tile 0 at [256, 384), of key tile 1 at [384, 512), fp32.
 // Shared memory (1024-aligned, 128-byte swizzle), default build:
-//   Q     = 2 d-halves x 256 rows x 128 B                   64 KB
-//   KV[5] = 5 x (K: 2 x 64 x 128 B, V: 2 x 64 x 128 B)     160 KB
+//   Q[2] = 2 x (2 d-halves x 128 rows x 128 B)              64 KB
+//   K[2] = 2 x (2 d-halves x 128 keys x 128 B)              64 KB
+//   V[2] = 2 x (2 tiles x 2 d-halves x 64 keys x 128 B)     64 KB
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
 namespace ft {
 
-#ifndef FVATTN_FT_STAGES
-#define FVATTN_FT_STAGES 5
+#ifndef FVATTN_FT_KSTAGES
+#define FVATTN_FT_KSTAGES 2
+#endif
+#ifndef FVATTN_FT_VSTAGES
+#define FVATTN_FT_VSTAGES 2
 #endif
 #ifndef FVATTN_FT_QBUF
-#define FVATTN_FT_QBUF 1
+#define FVATTN_FT_QBUF 2
 #endif
 constexpr int D = 128;
-constexpr int STAGES = FVATTN_FT_STAGES;   // K/V ring depth
+constexpr int KST = FVATTN_FT_KSTAGES;     // K ring depth
+constexpr int VST = FVATTN_FT_VSTAGES;     // V ring depth
 constexpr int QBUF = FVATTN_FT_QBUF;       // Q buffers (items in flight)
+constexpr int SBUF = 2;                    // TMEM S buffers
 constexpr int THREADS = 384;
 constexpr int SM_WARP0 = 4;                             // first softmax warp
 constexpr uint32_t BOX = 64 * 128;                      // one 64-row x 128-byte box: 8 KB
-constexpr uint32_t Q_BYTES = 8 * BOX;                   // 4 tiles x 2 d-halves: 64 KB
-constexpr uint32_t Q_HALF = 4 * BOX;                    // one d-half of the 256 Q rows
-constexpr uint32_t KV_TILE_BYTES = 2 * BOX;             // 16 KB
-constexpr uint32_t STAGE_BYTES = 2 * KV_TILE_BYTES;     // 32 KB
+constexpr uint32_t Q_BYTES = 4 * BOX;                   // 2 tiles x 2 d-halves: 32 KB
+constexpr uint32_t Q_HALF = 2 * BOX;                    // one d-half of the 128 Q rows
+constexpr uint32_t STAGE_BYTES = 4 * BOX;               // K or V of a step's two key tiles: 32 KB
+constexpr uint32_t K_HALF = 2 * BOX;                    // one d-half of the step's 128 keys
+constexpr uint32_t V_TILE = 2 * BOX;                    // one key tile of V (2 d-halves)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
+constexpr uint32_t TMEM_O = 256;                        // O of keys 0-31; keys 32-63 at +128
+constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, false, true);
-constexpr int ITEM_LAST = 1 << 24;
-
-struct Stream {
-  uint64_t s_full[2];     // S ready (MMA commit) + step info written (MMA thread arrive)
-  uint64_t p_full[2];     // P written by the 128 softmax threads
-  uint64_t pv_done[2];    // PV of step c completes pv_done[c & 1]; waiting on it by
-                          // parity is exact because the thread has already seen the
-                          // S commit that follows the PV of step c - 2
-  uint64_t o_empty;       // epilogue read O (128 arrivals per item)
-  int info[2];            // per S buffer: selection bits of this stream's two tiles | last << 2
-};
+constexpr int ENTRY_LAST = 1 << 22;   // union entry word: last entry of the item
+constexpr int STEP_LAST = 1 << 4;     // step word: sel of tile 0 (bits 0-1), tile 1 (bits 2-3), last
 
 struct Ctl {
   uint64_t q_full[QBUF], q_empty[QBUF];
-  uint64_t kv_full[STAGES], kv_empty[STAGES];
-  Stream st[2];
-  int meta[STAGES];
+  uint64_t k_full[KST], k_empty[KST];
+  uint64_t v_full[VST], v_empty[VST];
+  uint64_t s_full[SBUF];   // S ready (MMA commit) + step info written (MMA thread arrive)
+  uint64_t p_full[SBUF];   // both halves' P written (256 softmax threads)
+  uint64_t pv_done[SBUF];  // PV of step c complete: barrier c & 1, phase c >> 1 (the S of step
+                           // c waits for PV(c - 2), and PV(c + 2) needs P(c + 2), so a waiter
+                           // never sees two outstanding phases)
+  uint64_t o_empty;        // epilogue read both O (256 arrivals per item)
+  uint64_t xchg;           // epilogue (m, l) exchange between the halves (256 per item)
+  uint64_t drain;          // final commits of the two MMA threads
+  int info[SBUF];          // per S buffer: the step word
+  int meta[KST];
+  float xm[2][2][128], xl[2][2][128];   // [item parity][half][row]
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr uint32_t SMEM_BYTES = 1024 + QBUF * Q_BYTES + STAGES * STAGE_BYTES;
-// A row's running max may grow by this much (log2 units) before O is
-// rescaled: P is bf16 (exponent range 2^+-127) and O, l are fp32, so
-// probabilities up to 2^64 relative to the stale max are exact enough and
-// the rescale (a wait on the in-flight PV plus a TMEM read-modify-write of
-// O) almost never runs.
-constexpr float RESCALE_LOG2 = 64.f;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+constexpr uint32_t SMEM_BYTES = 1024 + QBUF * Q_BYTES + (KST + VST) * STAGE_BYTES;
+// A step whose probabilities (relative to the half-row's reference max) sum
+// past this bound triggers a rescale: P is bf16 (exponent range 2^+-127) and
+// O, l are fp32, so probabilities up to 2^64 are exact enough, and the
+// rescale (a wait on the in-flight PV plus a TMEM read-modify-write of O)
+// almost never runs.
+constexpr float RESCALE_SUM = 18446744073709551616.f;   // 2^64
+// Pairs of a key tile (32 pairs) whose exponentials use the polynomial.
+#ifndef FVATTN_FT_POLY_PAIRS
+#define FVATTN_FT_POLY_PAIRS 0
+#endif
+constexpr int POLY_PAIRS = FVATTN_FT_POLY_PAIRS;
+static_assert(POLY_PAIRS == 0 || POLY_PAIRS == 8 || POLY_PAIRS == 12 || POLY_PAIRS == 16, "poly split");
+__host__ __device__ constexpr bool poly_pair(int i) {
+  return POLY_PAIRS == 8 ? (i & 3) == 3
+       : POLY_PAIRS == 12 ? ((i & 7) == 1 || (i & 7) == 3 || (i & 7) == 6)
+       : POLY_PAIRS == 16 ? (i & 1) == 1 : false;
+}
+static_assert(SMEM_BYTES + sizeof(Ctl) <= 232448, "shared memory budget (dynamic + static)");
 
 }  // namespace ft
 
 // One 64-token tile of a [BH, N, 128] bf16 tensor: two 64-column boxes
-// (d 0-63 and 64-127) written `stride` bytes apart.
-__device__ inline void tma_tile(const CUtensorMap* map, int natural, const FineTcArgs& a, int bh, int tile,
-                                uint8_t* dst, uint32_t stride, uint64_t* bar) {
+// (d 0-63 and 64-127) written `stride` bytes apart.  `cube` is the tile's
+// packed cube coordinates (natural layout) and is unused for the tiled one.
+__device__ inline void tma_tile(const CUtensorMap* map, int natural, int cube, int bh, int tile, uint8_t* dst,
+                                uint32_t stride, uint64_t* bar) {
   if (natural) {
-    const int cube = a.tile_cube[tile];
     const int w0 = cube_w(cube) * 4, h0 = cube_h(cube) * 4, t0 = cube_t(cube) * 4;
     tma_load_5d(dst, map, bar, 0, w0, h0, t0, bh);
     tma_load_5d(dst + stride, map, bar, 64, w0, h0, t0, bh);
@@ -109,6 +138,128 @@ __device__ inline uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
+// Packed f32x2 helpers (sm_100 FFMA2 / FADD2).
+__device__ inline uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ inline void uf2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ inline uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ inline uint64_t add2_rm(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ inline uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ inline float max3f(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+// bf16x2 of (lo, hi), round to nearest even.
+__device__ inline uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// acc + the low / high bf16 half of w (exact widening, one fp32 rounding).
+__device__ inline float add_bf16_lo(float acc, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, l, %0;\n\t}" : "+f"(acc) : "r"(w));
+  return acc;
+}
+__device__ inline float add_bf16_hi(float acc, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %0;\n\t}" : "+f"(acc) : "r"(w));
+  return acc;
+}
+
+// 2^x for a pair on the FMA pipe (Cody-Waite style range reduction): x is
+// clamped to [-126, 126]; i = floor(x) comes from a round-down add of
+// 1.5 * 2^23 (the low mantissa bits of the sum hold i), f = x - i in [0, 1),
+// 2^f by a degree-3 polynomial, and i is added to the exponent field.  The
+// coefficients are a minimax fit of 2^f on [0, 1) in relative error, solved
+// as a linear program over a dense grid: max relative error 7.5e-5, below
+// half a bf16 ulp (2^-9), which is the precision P is stored in.
+__device__ inline void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float C0 = 0.9999252557754517f, C1 = 0.6958333253860474f, C2 = 0.22606715559959412f,
+                  C3 = 0.07802474498748779f, MAGIC = 12582912.f;
+  x0 = fminf(fmaxf(x0, -126.f), 126.f);
+  x1 = fminf(fmaxf(x1, -126.f), 126.f);
+  const uint64_t X = f2(x0, x1), M = f2(MAGIC, MAGIC);
+  const uint64_t Y = add2_rm(X, M);
+  const uint64_t F = sub2(X, sub2(Y, M));
+  uint64_t P = fma2(F, f2(C3, C3), f2(C2, C2));
+  P = fma2(P, F, f2(C1, C1));
+  P = fma2(P, F, f2(C0, C0));
+  float p0, p1, q0, q1;
+  uf2(P, p0, p1);
+  uf2(Y, q0, q1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(q0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(q1) << 23));
+}
+
+// Largest logit of a row's 64-key step.
+__device__ inline float row_max64(const uint32_t (&s0)[32], const uint32_t (&s1)[32]) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    m0 = max3f(m0, __uint_as_float(s0[i]), __uint_as_float(s0[i + 1]));
+    m1 = max3f(m1, __uint_as_float(s1[i]), __uint_as_float(s1[i + 1]));
+  }
+  return fmaxf(m0, m1);
+}
+
+// P = 2^(s * sl2 - m) of a row's 64-key step as 32 bf16x2 words (word k =
+// keys 2k, 2k+1); returns the sum of the bf16 values.
+__device__ inline float exp_step(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float sl2, float m,
+                                 uint32_t (&pk)[32]) {
+  const uint64_t SL = f2(sl2, sl2), NM = f2(-m, -m);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t* src = i < 16 ? s0 : s1;
+    const int j = 2 * (i & 15);
+    float x0, x1, p0, p1;
+    uf2(fma2(f2(__uint_as_float(src[j]), __uint_as_float(src[j + 1])), SL, NM), x0, x1);
+    if (ft::poly_pair(i)) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    const uint32_t w = cvt_bf16x2(p0, p1);
+    pk[i] = w;
+    if (i & 1) {
+      a2 = add_bf16_lo(a2, w);
+      a3 = add_bf16_hi(a3, w);
+    } else {
+      a0 = add_bf16_lo(a0, w);
+      a1 = add_bf16_hi(a1, w);
+    }
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __global__ void __launch_bounds__(ft::THREADS, 1)
     fine_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, const FineTcArgs a) {
@@ -116,7 +267,8 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + QBUF * Q_BYTES;
+  uint8_t* sK = sQ + QBUF * Q_BYTES;
+  uint8_t* sV = sK + KST * STAGE_BYTES;
   __shared__ Ctl ctl_s;
   Ctl* ctl = &ctl_s;
   volatile int* abort_flag = &ctl->abort;
@@ -127,21 +279,24 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < QBUF; ++i) {
       mbar_init(&ctl->q_full[i], 1);
-      mbar_init(&ctl->q_empty[i], 2);      // one release per stream
+      mbar_init(&ctl->q_empty[i], 1);
     }
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&ctl->kv_full[i], 1);
-      mbar_init(&ctl->kv_empty[i], 2);     // one release per stream
+    for (int i = 0; i < KST; ++i) {
+      mbar_init(&ctl->k_full[i], 1);
+      mbar_init(&ctl->k_empty[i], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&ctl->st[s].s_full[i], 2);
-        mbar_init(&ctl->st[s].p_full[i], 128);
-      }
-      mbar_init(&ctl->st[s].pv_done[0], 1);
-      mbar_init(&ctl->st[s].pv_done[1], 1);
-      mbar_init(&ctl->st[s].o_empty, 128);
+    for (int i = 0; i < VST; ++i) {
+      mbar_init(&ctl->v_full[i], 1);
+      mbar_init(&ctl->v_empty[i], 1);
     }
+    for (int i = 0; i < SBUF; ++i) {
+      mbar_init(&ctl->s_full[i], 2);
+      mbar_init(&ctl->p_full[i], 256);
+      mbar_init(&ctl->pv_done[i], 1);
+    }
+    mbar_init(&ctl->o_empty, 256);
+    mbar_init(&ctl->xchg, 256);
+    mbar_init(&ctl->drain, 2);           // one final commit per MMA thread
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -154,198 +309,251 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = ctl->tmem_base;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- TMA
-    prefetch_tensormap(&mq);
-    prefetch_tensormap(&mk);
-    prefetch_tensormap(&mv);
-    long long gs = 0;
-    int k = 0;
+    // The whole warp fetches the next 32 union entries (16 steps) and their
+    // cube coordinates with one pair of coalesced loads; lane 0 then issues
+    // the waits and copies step by step, so no copy waits on a global load.
+    const bool leader = lane == 0;
+    const bool nat = a.q_nat || a.k_nat || a.v_nat;
+    if (leader) {
+      prefetch_tensormap(&mq);
+      prefetch_tensormap(&mk);
+      prefetch_tensormap(&mv);
+    }
+    long long gs = 0;                 // steps loaded
+    int k = 0, q_issued = 0;
     bool ok = true;
+    int item_next = blockIdx.x < a.n_items ? a.worklist[blockIdx.x] : 0;
     for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
-      const int item = a.worklist[slot];
+      const int item = item_next;
+      if (slot + (int)gridDim.x < a.n_items) item_next = a.worklist[slot + gridDim.x];
       const int bh = item / g.P, qd = item % g.P;
       const int qb = k % QBUF;
-      if (k >= QBUF && !mbar_wait(&ctl->q_empty[qb], ((k / QBUF) - 1) & 1, abort_flag, a.status, cap)) break;
-      mbar_arrive_expect_tx(&ctl->q_full[qb], Q_BYTES);
-      uint8_t* qd_smem = sQ + qb * Q_BYTES;
-#pragma unroll 1
-      for (int t = 0; t < kItemTiles; ++t) {
-        int tile = kItemTiles * qd + t;
-        if (tile >= g.nT) tile = kItemTiles * qd;        // rows of a missing tile are never stored
-        tma_tile(&mq, a.q_nat, a, bh, tile, qd_smem + t * BOX, Q_HALF, &ctl->q_full[qb]);
-      }
+      // lanes 0, 1: the item's two query tiles (a missing second tile repeats the first; its rows
+      // are never stored)
+      int qtile = kItemTiles * qd + (lane & 1);
+      if (qtile >= g.nT) qtile = kItemTiles * qd;
+      const int qcube = nat && lane < kItemTiles ? a.tile_cube[qtile] : 0;
       const int n = a.ucount[item];
       const int* list = a.uni + (size_t)item * g.nT;
-      int next = list[0];
-      for (int e = 0; e < n; ++e, ++gs) {
-        int ent = next;
-        if (e + 1 < n) next = list[e + 1];
-        const int st = (int)(gs % STAGES);
-        if (gs >= STAGES &&
-            !mbar_wait(&ctl->kv_empty[st], (uint32_t)((gs / STAGES) - 1) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
+      if (leader && k >= QBUF) ok = mbar_wait(&ctl->q_empty[qb], ((k / QBUF) - 1) & 1, abort_flag, a.status, cap);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int qc0 = __shfl_sync(0xffffffffu, qcube, 0), qc1 = __shfl_sync(0xffffffffu, qcube, 1);
+      const int qt0 = __shfl_sync(0xffffffffu, qtile, 0), qt1 = __shfl_sync(0xffffffffu, qtile, 1);
+      if (leader) {
+        mbar_arrive_expect_tx(&ctl->q_full[qb], Q_BYTES);
+        uint8_t* qd_smem = sQ + qb * Q_BYTES;
+        tma_tile(&mq, a.q_nat, qc0, bh, qt0, qd_smem, Q_HALF, &ctl->q_full[qb]);
+        tma_tile(&mq, a.q_nat, qc1, bh, qt1, qd_smem + BOX, Q_HALF, &ctl->q_full[qb]);
+      }
+      ++q_issued;
+      const int steps = (n + 1) >> 1;
+      for (int e0 = 0; e0 < n && ok; e0 += 32) {
+        int ent = e0 + lane < n ? list[e0 + lane] : 0;
         int j = ent & 0xFFFF;
         if (j >= g.nT) {  // never produced by the schedule; keep the copy in bounds
           set_status(a.status, kStatusBadBlock);
           j = 0;
-          ent &= ~0xF0000;
+          ent &= ~0x30000;
         }
-        ctl->meta[st] = ent | (e == n - 1 ? ITEM_LAST : 0);
-        mbar_arrive_expect_tx(&ctl->kv_full[st], STAGE_BYTES);
-        uint8_t* kd = sKV + st * STAGE_BYTES;
-        tma_tile(&mk, a.k_nat, a, bh, j, kd, BOX, &ctl->kv_full[st]);
-        tma_tile(&mv, a.v_nat, a, bh, j, kd + KV_TILE_BYTES, BOX, &ctl->kv_full[st]);
+        const int cube = nat ? a.tile_cube[j] : 0;
+        const int cnt = n - e0 < 32 ? n - e0 : 32;
+        for (int i = 0; i < cnt; i += 2, ++gs) {
+          // the step's key tiles: entries e0 + i and e0 + i + 1 (a masked copy of the first when
+          // the item's entry count is odd)
+          const bool two = i + 1 < cnt;
+          const int ent0 = __shfl_sync(0xffffffffu, ent, i);
+          const int cube0 = __shfl_sync(0xffffffffu, cube, i);
+          const int ent1 = __shfl_sync(0xffffffffu, ent, two ? i + 1 : i);
+          const int cube1 = __shfl_sync(0xffffffffu, cube, two ? i + 1 : i);
+          if (leader) {
+            const int j0 = ent0 & 0xFFFF, j1 = ent1 & 0xFFFF;
+            const int ks = (int)(gs % KST), vs = (int)(gs % VST);
+            const int step = (e0 + i) >> 1;
+            if (gs >= KST)
+              ok = mbar_wait(&ctl->k_empty[ks], (uint32_t)((gs / KST) - 1) & 1, abort_flag, a.status, cap);
+            if (ok) {
+              ctl->meta[ks] = ((ent0 >> 16) & 3) | (two ? ((ent1 >> 16) & 3) << 2 : 0) |
+                              (step == steps - 1 ? STEP_LAST : 0);
+              mbar_arrive_expect_tx(&ctl->k_full[ks], STAGE_BYTES);
+              uint8_t* kd = sK + ks * STAGE_BYTES;
+              tma_tile(&mk, a.k_nat, cube0, bh, j0, kd, K_HALF, &ctl->k_full[ks]);
+              tma_tile(&mk, a.k_nat, cube1, bh, j1, kd + BOX, K_HALF, &ctl->k_full[ks]);
+              if (gs >= VST)
+                ok = mbar_wait(&ctl->v_empty[vs], (uint32_t)((gs / VST) - 1) & 1, abort_flag, a.status, cap);
+            }
+            if (ok) {
+              mbar_arrive_expect_tx(&ctl->v_full[vs], STAGE_BYTES);
+              uint8_t* vd = sV + vs * STAGE_BYTES;
+              tma_tile(&mv, a.v_nat, cube0, bh, j0, vd, BOX, &ctl->v_full[vs]);
+              tma_tile(&mv, a.v_nat, cube1, bh, j1, vd + V_TILE, BOX, &ctl->v_full[vs]);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+        }
       }
     }
-  } else if ((warp == 1 || warp == 2) && lane == 0) {
-    // ------------------------------------------------- MMA (one per stream)
-    // Stream x's issuer walks every entry in order.  Entries it takes part
-    // in: S of step c into S buffer c & 1, then the PV of step c - 1 once its
-    // P is written (so the softmax always has the next S ready).  Entries it
-    // sits out: it settles any pending PV and releases its share of the
-    // stage.  A stage is reloaded once both streams released it; a Q buffer
-    // once both issuers passed the item's last entry.
-    const int x = warp - 1;
-    Stream& S = ctl->st[x];
-    const uint64_t qdesc0 = umma_desc_sw128(smem_u32(sQ), 16, 1024) + (uint64_t)((x * 2 * BOX) >> 4);
-    const uint64_t kdesc0 = umma_desc_sw128(smem_u32(sKV), 16, 1024);
-    const uint64_t vdesc0 = umma_desc_sw128(smem_u32(sKV + KV_TILE_BYTES), BOX, 1024);
-    const uint32_t tS0 = tbase + 256 * x, tO = tbase + 256 * x + 128;
-    long long gs = 0, c = 0;
+    // every copy issued has landed before the block exits
+    if (leader) {
+      for (int qb = 0; qb < QBUF && qb < q_issued; ++qb) {
+        const int last = qb + ((q_issued - 1 - qb) / QBUF) * QBUF;
+        mbar_drain(&ctl->q_full[qb], (uint32_t)(last / QBUF) & 1, a.status, cap);
+      }
+      for (int i = 0; i < KST && i < gs; ++i) {
+        const long long last = i + ((gs - 1 - i) / KST) * KST;
+        mbar_drain(&ctl->k_full[i], (uint32_t)(last / KST) & 1, a.status, cap);
+      }
+      for (int i = 0; i < VST && i < gs; ++i) {
+        const long long last = i + ((gs - 1 - i) / VST) * VST;
+        mbar_drain(&ctl->v_full[i], (uint32_t)(last / VST) & 1, a.status, cap);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------- MMA: S
+    // S(c) into buffer c & 1 once the PV of step c - 2, which read its P
+    // from that buffer, is complete; a K stage is released when its S
+    // completes, the Q buffer after the item's last S.
+    long long c = 0;
     int k = 0;
-    bool pend = false, pend_first = false, ok = true;
-    long long pend_c = 0;
-    int pend_stage = 0, pend_item = 0;
-    auto issue_pv = [&]() -> bool {
-      const int b = (int)(pend_c & 1);
-      if (!mbar_wait(&S.p_full[b], (uint32_t)(pend_c >> 1) & 1, abort_flag, a.status, cap)) return false;
-      if (pend_first && pend_item >= 1 &&
-          !mbar_wait(&S.o_empty, (uint32_t)(pend_item - 1) & 1, abort_flag, a.status, cap))
-        return false;
-      tc_fence_after();
-      const uint64_t vd = vdesc0 + (uint64_t)((pend_stage * STAGE_BYTES) >> 4);
-      const uint32_t tP = tS0 + 64 * b;
-      mma_ts(tO, tP, vd, IDESC_PV, pend_first ? 0u : 1u);
-#pragma unroll
-      for (int kk = 1; kk < 4; ++kk) mma_ts(tO, tP + kk * 8, vd + kk * (2048 >> 4), IDESC_PV, 1u);
-      mma_commit(&S.pv_done[b]);
-      mma_commit(&ctl->kv_empty[pend_stage]);
-      pend = false;
-      return true;
-    };
+    bool ok = true;
     for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
       const int qb = k % QBUF;
       if (!mbar_wait(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
-      const uint64_t qd = qdesc0 + (uint64_t)((qb * Q_BYTES) >> 4);
-      bool first = true;
+      const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
       while (true) {
-        const int st = (int)(gs % STAGES);
-        if (!mbar_wait(&ctl->kv_full[st], (uint32_t)(gs / STAGES) & 1, abort_flag, a.status, cap)) {
+        const int ks = (int)(c % KST);
+        const int b = (int)(c & 1);
+        // K first: it is loaded well ahead, the PV wait is the one on the critical path
+        if (!mbar_wait(&ctl->k_full[ks], (uint32_t)(c / KST) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
-        const int meta = ctl->meta[st];
-        if ((meta >> (20 + x)) & 1) {
-          const int b = (int)(c & 1);
-          S.info[b] = ((meta >> (16 + 2 * x)) & 3) | (((meta >> (22 + x)) & 1) << 2);
-          tc_fence_after();
-          const uint64_t kd = kdesc0 + (uint64_t)((st * STAGE_BYTES) >> 4);
-          const uint32_t tS = tS0 + 64 * b;
-          mma_ss(tS, qd, kd, IDESC_S, 0u);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            mma_ss(tS, qd + (((kk >> 2) * Q_HALF + (kk & 3) * 32) >> 4), kd + (((kk >> 2) * BOX + (kk & 3) * 32) >> 4),
-                   IDESC_S, 1u);
-          mma_commit(&S.s_full[b]);
-          mbar_arrive(&S.s_full[b]);
-          if (pend && !issue_pv()) {
-            ok = false;
-            break;
-          }
-          pend = true;
-          pend_c = c;
-          pend_stage = st;
-          pend_first = first;
-          pend_item = k;
-          first = false;
-          ++c;
-        } else {
-          if (pend && !issue_pv()) {
-            ok = false;
-            break;
-          }
-          mbar_arrive(&ctl->kv_empty[st]);
+        if (c >= SBUF && !mbar_wait(&ctl->pv_done[b], (uint32_t)((c - SBUF) >> 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
         }
-        ++gs;
-        if (meta & ITEM_LAST) break;
+        const int meta = ctl->meta[ks];
+        ctl->info[b] = meta;
+        tc_fence_after();
+        const uint64_t kd = umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024);
+        const uint32_t tS = tbase + 128 * b;
+        mma_ss(tS, qd, kd, IDESC_S, 0u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          mma_ss(tS, qd + (((kk >> 2) * Q_HALF + (kk & 3) * 32) >> 4),
+                 kd + (((kk >> 2) * K_HALF + (kk & 3) * 32) >> 4), IDESC_S, 1u);
+        mma_commit(&ctl->s_full[b]);
+        mma_commit(&ctl->k_empty[ks]);
+        mbar_arrive(&ctl->s_full[b]);
+        ++c;
+        if (meta & STEP_LAST) break;
       }
       if (!ok) break;
       mma_commit(&ctl->q_empty[qb]);
     }
-    if (ok && pend) issue_pv();
+    // every MMA this thread issued has completed before TMEM is freed
+    mma_commit(&ctl->drain);
+    mbar_drain(&ctl->drain, 0, a.status, cap);
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------------------ MMA: PV
+    // O_t += P_t V_t for the step's key tiles t = 0, 1 once both softmax
+    // groups wrote P; the first step of an item overwrites O after the
+    // previous item's epilogue read it.  A V stage is released when its PV
+    // completes.
+    long long c = 0;
+    int k = 0;
+    bool ok = true;
+    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+      bool first = true;
+      while (true) {
+        const int b = (int)(c & 1);
+        const int vs = (int)(c % VST);
+        // O free and V loaded come well before P, the wait on the critical path
+        if (first && k >= 1 && !mbar_wait(&ctl->o_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&ctl->v_full[vs], (uint32_t)(c / VST) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&ctl->p_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        const int info = ctl->info[b];
+        tc_fence_after();
+        const uint32_t tP = tbase + 128 * b;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint64_t vd = umma_desc_sw128(smem_u32(sV + vs * STAGE_BYTES + t * V_TILE), BOX, 1024);
+          const uint32_t tO = tbase + TMEM_O + 128 * t;
+          // 16 keys = 16 V rows = 2048 bytes per K step; P of tile t in columns 64 t .. 64 t + 31
+          mma_ts(tO, tP + 64 * t, vd, IDESC_PV, first ? 0u : 1u);
+#pragma unroll
+          for (int kk = 1; kk < 4; ++kk) mma_ts(tO, tP + 64 * t + 8 * kk, vd + ((kk * 2048) >> 4), IDESC_PV, 1u);
+        }
+        mma_commit(&ctl->pv_done[b]);
+        mma_commit(&ctl->v_empty[vs]);
+        first = false;
+        ++c;
+        if (info & STEP_LAST) break;
+      }
+    }
+    mma_commit(&ctl->drain);
+    mbar_drain(&ctl->drain, 0, a.status, cap);
   } else if (warp >= SM_WARP0) {
     // ------------------------------------------------------------ softmax
-    const int s = (warp - SM_WARP0) >> 2;             // stream
-    Stream& S = ctl->st[s];
+    const int h = (warp - SM_WARP0) >> 2;             // key tile of every step
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;                     // row of the stream
-    const int half = r >> 6, rr = r & 63;
+    const int r = q4 * 32 + lane;                     // row of the item
+    const int half = r >> 6, rr = r & 63;             // query tile of the row, row in it
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tcol = tbase + 256 * s;
-    const uint32_t tO = tcol + 128 + lane_off;
+    const uint32_t tO = tbase + TMEM_O + 128 * h + lane_off;
     const float sl2 = g.scale * 1.4426950408889634f;
     long long c = 0;
-    for (int slot = blockIdx.x; slot < a.n_items; slot += gridDim.x) {
-      const int item = a.worklist[slot];
+    int k = 0;
+    int item_next = blockIdx.x < a.n_items ? a.worklist[blockIdx.x] : 0;
+    for (int slot = blockIdx.x; slot < a.n_items; slot += gridDim.x, ++k) {
+      const int item = item_next;                     // the next item's code loads during this one
+      if (slot + (int)gridDim.x < a.n_items) item_next = a.worklist[slot + gridDim.x];
       const int bh = item / g.P, qd = item % g.P;
-      const int tile = kItemTiles * qd + 2 * s + half;
+      const int tile = kItemTiles * qd + half;
       const bool valid = tile < g.nT;
+      const int cube = valid && a.out_nat ? a.tile_cube[tile] : 0;   // used by the epilogue
       float m_use = -INFINITY, l = 0.f;
       bool ok = true;
       while (true) {
-        const int sb = (int)(c & 1);
-        if (!mbar_wait(&S.s_full[sb], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+        const int b = (int)(c & 1);
+        if (!mbar_wait(&ctl->s_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int info = S.info[sb];
-        const bool sel = (info >> half) & 1;
-        const uint32_t tSrow = tcol + 64 * sb + lane_off;
+        const int info = ctl->info[b];
+        const bool sel = (info >> (2 * h + half)) & 1;
+        const uint32_t tS = tbase + 128 * b + 64 * h + lane_off;
         uint32_t pk[32];
         float alpha = 1.f;
         bool rescale = false;
         {
           uint32_t s0[32], s1[32];
-          tmem_ld32(tSrow, s0);
-          tmem_ld32(tSrow + 32, s1);
+          tmem_ld32(tS, s0);
+          tmem_ld32(tS + 32, s1);
           tmem_wait_ld();
           if (sel) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(__uint_as_float(s0[i]), __uint_as_float(s1[i])));
-            const float m_new = mx * sl2;
-            if (m_new > m_use + RESCALE_LOG2) {
+            if (m_use == -INFINITY) m_use = row_max64(s0, s1) * sl2;   // first selected tile of the row
+            float sum = exp_step(s0, s1, sl2, m_use, pk);
+            if (!(sum <= RESCALE_SUM)) {      // too large (or inf): move the reference max up
+              const float m_new = fmaxf(row_max64(s0, s1) * sl2, m_use);
               alpha = ex2(m_use - m_new);
               rescale = l > 0.f;
               l *= alpha;
               m_use = m_new;
-            }
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = ex2(fmaf(__uint_as_float(s0[2 * i]), sl2, -m_use));
-              const float p1 = ex2(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, -m_use));
-              const float p2 = ex2(fmaf(__uint_as_float(s1[2 * i]), sl2, -m_use));
-              const float p3 = ex2(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, -m_use));
-              pk[i] = pack_bf16(p0, p1);
-              pk[16 + i] = pack_bf16(p2, p3);
-              // normalise with the probabilities as the MMA sees them (bf16)
-              sum += (__uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u)) +
-                     (__uint_as_float(pk[16 + i] << 16) + __uint_as_float(pk[16 + i] & 0xFFFF0000u));
+              sum = exp_step(s0, s1, sl2, m_use, pk);
             }
             l += sum;
           } else {
@@ -353,9 +561,10 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
             for (int i = 0; i < 32; ++i) pk[i] = 0u;
           }
         }
-        tmem_st32(tSrow, pk);
+        tmem_st32(tS, pk);
         if (__any_sync(0xffffffffu, rescale)) {
-          if (!mbar_wait(&S.pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) {
+          // O must hold every PV before step c; PV(c) waits for this step's P
+          if (!mbar_wait(&ctl->pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) {
             ok = false;
             break;
           }
@@ -372,36 +581,51 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&S.p_full[sb]);
+        mbar_arrive(&ctl->p_full[b]);
         ++c;
-        if (info & 4) break;
+        if (info & STEP_LAST) break;
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> out, lse
-      if (!mbar_wait(&S.pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) break;
+      // ---- epilogue: merge the groups' (m, l, O); this group writes dims 64 h .. 64 h + 63
+      if (!mbar_wait(&ctl->pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) break;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int tok = !valid ? 0 : (a.out_nat ? cube_row_token(g, a.tile_cube[tile], rr) : tile * kTileTokens + rr);
-      __nv_bfloat16* orow = a.out + ((size_t)bh * g.N + tok) * D;
+      const int kp = k & 1;
+      ctl->xm[kp][h][r] = m_use;
+      ctl->xl[kp][h][r] = l;
+      mbar_arrive(&ctl->xchg);
+      if (!mbar_wait(&ctl->xchg, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
+      const float m0 = ctl->xm[kp][0][r], m1 = ctl->xm[kp][1][r];
+      const float l0 = ctl->xl[kp][0][r], l1 = ctl->xl[kp][1][r];
+      const float M = fmaxf(m0, m1);
+      const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+      const float w1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+      const float L = l0 * w0 + l1 * w1;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float s0 = w0 * inv, s1 = w1 * inv;
+      const int tok = !valid ? 0 : (a.out_nat ? cube_row_token(g, cube, rr) : tile * kTileTokens + rr);
+      __nv_bfloat16* orow = a.out + ((size_t)bh * g.N + tok) * D + 64 * h;
+      const uint32_t tO0 = tbase + TMEM_O + lane_off + 64 * h, tO1 = tO0 + 128;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t o[32];
-        tmem_ld32(tO + ch * 32, o);
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + ch * 32, o0);
+        tmem_ld32(tO1 + ch * 32, o1);
         tmem_wait_ld();
         if (valid) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            w[i] = pack_bf16(__uint_as_float(o0[2 * i]) * s0 + __uint_as_float(o1[2 * i]) * s1,
+                             __uint_as_float(o0[2 * i + 1]) * s0 + __uint_as_float(o1[2 * i + 1]) * s1);
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (valid)
-        a.lse[(size_t)bh * g.N + tok] = l > 0.f ? (m_use + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (valid && h == 0)
+        a.lse[(size_t)bh * g.N + tok] = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
       tc_fence_before();
-      mbar_arrive(&S.o_empty);
+      mbar_arrive(&ctl->o_empty);
     }
   }
 

@@ -15,7 +15,7 @@
 namespace fvattn {
 
 constexpr int kTileTokens = 64;
-constexpr int kItemTiles = 4;   // query tiles per fine-stage work item (two 128-row streams)
+constexpr int kItemTiles = 2;   // query tiles per fine-stage work item (one 128-row tile)
 constexpr int kMaxTiles = 8192;
 
 // Device status codes (workspace status word).
@@ -134,6 +134,12 @@ __device__ inline uint32_t smem_u32(const void* p) {
 
 __device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tcgen05.mma operands) before a release that hands them over.
+__device__ inline void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ inline void fence_mbar_init() {

@@ -2,38 +2,35 @@
 // runtime head-level load balancing (section 02), applied across the SMs of
 // one GPU instead of across GPUs.
 //
-// A work item is four adjacent query tiles 4q .. 4q+3 of one (batch, head):
-// two 128-row tensor-core streams, A = tiles (4q, 4q+1) and B = tiles
-// (4q+2, 4q+3), that share every K/V tile the item loads.  The item walks
-// the union of the four tiles' key lists; each entry records which of the
-// four tiles selected it (the other tiles' rows are masked for it), which
-// stream takes part in it, and each stream's last entry.  Items are ranked by
-// union size, longest first (LPT), ties by item code, so the persistent fine
-// kernel hands the heavy items out first and the light ones fill the tail.
+// A work item is two adjacent query tiles 2q, 2q+1 of one (batch, head): one
+// 128-row tensor-core tile.  The item walks the union of the two tiles' key
+// lists; each entry records which of the two tiles selected it (the other
+// tile's rows are masked for it).  Items are ranked by union size, longest
+// first (LPT), ties by item code, so the persistent fine kernel hands the
+// heavy items out first and the light ones fill the tail.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
 
 // Entry word of the union list.
 //   bits  0-15  key tile id
-//   bits 16-19  selected by tile 4q+0 .. 4q+3
-//   bits 20-21  stream A / B takes part (a selecting tile, or the stream's
-//               one forced step when none of its tiles selected anything)
-//   bits 22-23  last entry of stream A / B in this item
-// One warp per item.  Validates the lists: counts in [0, nT], ids in
-// [0, nT) and strictly ascending; violations set kStatusBadBlock and the
-// offending entries are dropped.
+//   bits 16-17  selected by tile 2q / 2q+1
+//   bit     22  last entry of the item
+// An item none of whose tiles selected anything gets one fully masked entry
+// (its rows end with out = 0, lse = -inf).  One warp per item.  Validates
+// the lists: counts in [0, nT], ids in [0, nT) and strictly ascending;
+// violations set kStatusBadBlock and the offending entries are dropped.
 __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restrict__ counts,
                                                     const int* __restrict__ idx, int cap, int* __restrict__ uni,
                                                     int* __restrict__ ucount, int* status) {
-  extern __shared__ uint32_t bm[];  // per warp: 4 bitmaps of ceil(nT/32) words
+  extern __shared__ uint32_t bm[];  // per warp: kItemTiles bitmaps of ceil(nT/32) words
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int words = (g.nT + 31) / 32;
-  uint32_t* bmw = bm + warp * 4 * words;
+  uint32_t* bmw = bm + warp * kItemTiles * words;
   const long long item = (long long)blockIdx.x * 4 + warp;
   if (item >= (long long)g.BH * g.P) return;
   const int bh = (int)(item / g.P), qd = (int)(item % g.P);
-  for (int w = lane; w < 4 * words; w += 32) bmw[w] = 0u;
+  for (int w = lane; w < kItemTiles * words; w += 32) bmw[w] = 0u;
   __syncwarp();
   for (int t = 0; t < kItemTiles; ++t) {
     const int tile = kItemTiles * qd + t;
@@ -58,38 +55,24 @@ __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restric
   }
   __syncwarp();
   int* out = uni + item * (long long)g.nT;
-  int n = 0, lastA = -1, lastB = -1;
+  int n = 0;
   for (int w = 0; w < words; ++w) {
     const int j = w * 32 + lane;
     uint32_t sel = 0;
 #pragma unroll
     for (int t = 0; t < kItemTiles; ++t) sel |= ((bmw[t * words + w] >> lane) & 1u) << t;
-    const uint32_t part = ((sel & 3u) ? 1u : 0u) | ((sel & 12u) ? 2u : 0u);
     const unsigned bal = __ballot_sync(0xffffffffu, sel != 0u);
     const int pos = n + __popc(bal & ((1u << lane) - 1u));
-    if (sel) out[pos] = j | (int)(sel << 16) | (int)(part << 20);
-    const unsigned ba = __ballot_sync(0xffffffffu, (part & 1u) != 0u);
-    const unsigned bb = __ballot_sync(0xffffffffu, (part & 2u) != 0u);
-    if (ba) lastA = n + __popc(bal & ((2u << (31 - __clz(ba))) - 1u)) - 1;
-    if (bb) lastB = n + __popc(bal & ((2u << (31 - __clz(bb))) - 1u)) - 1;
+    if (sel) out[pos] = j | (int)(sel << 16);
     n += __popc(bal);
   }
   __syncwarp();
   if (lane == 0) {
-    if (n == 0) {  // no tile selected anything: one step, fully masked, for both streams
+    if (n == 0) {  // no tile selected anything: one fully masked step
       out[0] = 0;
       n = 1;
     }
-    if (lastA < 0) {  // stream A without a selection: it takes part in entry 0, masked
-      out[0] |= 1 << 20;
-      lastA = 0;
-    }
-    if (lastB < 0) {
-      out[0] |= 1 << 21;
-      lastB = 0;
-    }
-    out[lastA] |= 1 << 22;
-    out[lastB] |= 1 << 23;
+    out[n - 1] |= 1 << 22;
     ucount[item] = n;
   }
 }
@@ -126,7 +109,7 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
                          cudaStream_t s) {
   const long long items = (long long)g.BH * g.P;
   const int words = (g.nT + 31) / 32;
-  const size_t smem = (size_t)4 * 4 * words * sizeof(uint32_t);
+  const size_t smem = (size_t)4 * kItemTiles * words * sizeof(uint32_t);
   union_kernel<<<(unsigned)((items + 3) / 4), 128, smem, s>>>(g, counts, idx, cap, uni, ucount, status);
   return cudaGetLastError();
 }

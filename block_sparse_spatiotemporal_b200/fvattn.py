@@ -226,7 +226,7 @@ def _blocks_of(counts, idx):
 
 
 def build_worklist(shape: Shape, counts, idx, ws, stream=None):
-    P = (num_tiles(shape) + 3) // 4
+    P = (num_tiles(shape) + 1) // 2
     wl = torch.empty(shape.batch * shape.heads * P, dtype=torch.int32, device=counts.device)
     b = _blocks_of(counts, idx)
     _check("fvattn_build_worklist", lib().fvattn_build_worklist(ctypes.byref(shape), ctypes.byref(b), _ptr(wl),

@@ -155,10 +155,10 @@ int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void* q, const v
                                const fvattn_blocks* out, fvattn_stream_t stream);
 
 /* Schedule of the fine stage (single-GPU analogue of the "FVAttn" digest's
- * runtime head-level load balancing, section 02): a work item is four
- * adjacent query tiles 4q .. 4q+3 of one (batch, head), encoded
- * ((b*H + h)*P + q) with P = ceil(nT/4); its cost is the size of the union
- * of the four tiles' lists (tiles past nT contribute nothing); items are
+ * runtime head-level load balancing, section 02): a work item is two
+ * adjacent query tiles 2q, 2q+1 of one (batch, head), encoded
+ * ((b*H + h)*P + q) with P = ceil(nT/2); its cost is the size of the union
+ * of the two tiles' lists (a tile past nT contributes nothing); items are
  * sorted by cost descending, ties by ascending item code
  * (longest-processing-time first).  worklist has B*H*P int32. */
 int fvattn_build_worklist(const fvattn_shape* shape, const fvattn_blocks* blocks,

@@ -139,7 +139,7 @@ def _fine_case(wl, layout, top_p=None, k_min=None):
 
 @pytest.mark.parametrize("case", [
     dict(grid=(8, 16, 16), dtype="f32", d=64, gen="fixed", top_p=0.9, k_min=2),
-    dict(grid=(4, 8, 8), dtype="bf16", d=128, top_p=1.0, k_min=1),                 # dense, one item
+    dict(grid=(4, 8, 8), dtype="bf16", d=128, top_p=1.0, k_min=1),                 # dense, two items
     dict(grid=(4, 4, 12), dtype="bf16", d=128, top_p=1.0, k_min=1),                # odd nT: single-tile item
     dict(grid=(8, 16, 16), dtype="bf16", d=128, top_p=0.9, k_min=2),
     dict(grid=(8, 16, 16), dtype="bf16", d=128, top_p=0.0, k_min=5),               # fixed top-k
@@ -193,9 +193,9 @@ def test_empty_rows_and_bad_block_ids():
 
 
 def test_worklist_is_longest_union_first():
-    wl = small((8, 8, 20), heads=4)         # nT = 20 tiles: 5 items per head
+    wl = small((8, 8, 20), heads=4)         # nT = 20 tiles: 10 items per head
     _worklist_case(wl)
-    _worklist_case(small((4, 8, 20), heads=3))   # nT = 10: the last item has 2 tiles
+    _worklist_case(small((4, 4, 12), heads=3))   # nT = 3: the last item has one tile
 
 
 def _worklist_case(wl):
@@ -207,12 +207,12 @@ def _worklist_case(wl):
     oi = np.stack([r["idx"] for r in res])[None].astype(np.int32)
     cd, idd = torch.from_numpy(oc).cuda(), torch.from_numpy(oi).cuda()
     got = F.build_worklist(shape, cd, idd, ws).cpu().numpy()
-    P = (nT + 3) // 4
+    P = (nT + 1) // 2
     cost = []
     for h, r in enumerate(res):
         for p in range(P):
             u = set()
-            for t in range(4 * p, min(4 * p + 4, nT)):
+            for t in range(2 * p, min(2 * p + 2, nT)):
                 u |= set(r["idx"][t, :r["counts"][t]].tolist())
             cost.append(len(u))
     cost = np.array(cost)
