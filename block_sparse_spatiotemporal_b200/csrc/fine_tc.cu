@@ -5,9 +5,9 @@
 // Persistent kernel, one CTA per SM, 384 threads.  A work item is two
 // adjacent query tiles of one head: one 128-row tensor-core tile walking the
 // union of the two tiles' key lists two entries (128 keys) per step.
-//   warp 0       TMA producer: the item's Q (double-buffered across items),
-//                K and V of every step's two key tiles into 2-stage rings
-//                (a load has about one softmax step of lead);
+//   warp 0       TMA producer: the item's Q, K of every step's two key
+//                tiles into a 2-stage ring and V into a 3-stage ring (V is
+//                consumed last, so its ring is the deeper one);
 //   warp 1       S issuer (one thread): S = Q K^T (M=128, N=128, K=128) of
 //                step c into TMEM S buffer c & 1 once the PV of step c - 2
 //                (the buffer's previous P) is complete;
@@ -34,9 +34,9 @@
 // columns 64 t .. 64 t + 63 (its P, bf16, overwrites the first 32); O of
 // key tile 0 at [256, 384), of key tile 1 at [384, 512), fp32.
 // Shared memory (1024-aligned, 128-byte swizzle), default build:
-//   Q[2] = 2 x (2 d-halves x 128 rows x 128 B)              64 KB
+//   Q    = 2 d-halves x 128 rows x 128 B                    32 KB
 //   K[2] = 2 x (2 d-halves x 128 keys x 128 B)              64 KB
-//   V[2] = 2 x (2 tiles x 2 d-halves x 64 keys x 128 B)     64 KB
+//   V[3] = 3 x (2 tiles x 2 d-halves x 64 keys x 128 B)     96 KB
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
@@ -46,10 +46,10 @@ namespace ft {
 #define FVATTN_FT_KSTAGES 2
 #endif
 #ifndef FVATTN_FT_VSTAGES
-#define FVATTN_FT_VSTAGES 2
+#define FVATTN_FT_VSTAGES 3
 #endif
 #ifndef FVATTN_FT_QBUF
-#define FVATTN_FT_QBUF 2
+#define FVATTN_FT_QBUF 1
 #endif
 constexpr int D = 128;
 constexpr int KST = FVATTN_FT_KSTAGES;     // K ring depth
@@ -85,11 +85,15 @@ struct Ctl {
   uint64_t drain;          // final commits of the two MMA threads
   int info[SBUF];          // per S buffer: the step word
   int meta[KST];
-  float xm[2][2][128], xl[2][2][128];   // [item parity][half][row]
+  float xm[2][128], xl[2][128];   // epilogue exchange [group][row] (a group rewrites its slot only
+                                  // after the other group's P of the next step, so after its read)
   uint32_t tmem_base;
   int abort;
 };
 
+// The 128-byte swizzle atoms of TMA and UMMA need 1024-byte alignment: the
+// kernel rounds its dynamic shared-memory base up inside a 1 KB larger
+// allocation.
 constexpr uint32_t SMEM_BYTES = 1024 + QBUF * Q_BYTES + (KST + VST) * STAGE_BYTES;
 // A step whose probabilities (relative to the half-row's reference max) sum
 // past this bound triggers a rescale: P is bf16 (exponent range 2^+-127) and
@@ -589,13 +593,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       // ---- epilogue: merge the groups' (m, l, O); this group writes dims 64 h .. 64 h + 63
       if (!mbar_wait(&ctl->pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) break;
       tc_fence_after();
-      const int kp = k & 1;
-      ctl->xm[kp][h][r] = m_use;
-      ctl->xl[kp][h][r] = l;
+      ctl->xm[h][r] = m_use;
+      ctl->xl[h][r] = l;
       mbar_arrive(&ctl->xchg);
       if (!mbar_wait(&ctl->xchg, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
-      const float m0 = ctl->xm[kp][0][r], m1 = ctl->xm[kp][1][r];
-      const float l0 = ctl->xl[kp][0][r], l1 = ctl->xl[kp][1][r];
+      const float m0 = ctl->xm[0][r], m1 = ctl->xm[1][r];
+      const float l0 = ctl->xl[0][r], l1 = ctl->xl[1][r];
       const float M = fmaxf(m0, m1);
       const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
       const float w1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);

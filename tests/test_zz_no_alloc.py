@@ -53,7 +53,7 @@ def test_noalloc_pool_select_matches_workspace_entry_point():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    big = F.make_shape(1, 40, 128, (20, 32, 52))         # needs 82.5 MiB of scratch
+    big = F.make_shape(1, 40, 128, (20, 32, 52))         # needs 144 MiB of scratch
     x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     _, _, blocks = F.new_blocks(F.make_shape(1, 1, 128, (4, 4, 4)))
     st = F.lib().fvattn_pool_select_noalloc(ctypes.byref(big), ctypes.c_void_p(x.data_ptr()),
