@@ -309,6 +309,25 @@ def run_gpu(args, wl):
         e2e = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # ---- the tile reorder as its own pass (the forward folds it into its loads): q, k, v to
+    # tiled layout and out back, 2 bytes moved per byte
+    tmp = torch.empty_like(qd)
+    for _ in range(2):
+        F.tile_reorder(shape, qd, ws, out=tmp)
+    torch.cuda.synchronize(dev)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_reo = 5
+    r0.record(stream)
+    for _ in range(n_reo):
+        for x in (qd, kd, vd):
+            F.tile_reorder(shape, x, ws, out=tmp)
+        F.tile_reorder(shape, out, ws, inverse=True, out=tmp)
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    reorder_ms = r0.elapsed_time(r1) / n_reo
+    reorder_bytes = 4 * 2 * qd.numel() * qd.element_size()
+    del tmp
+
     if rank == 0:
         pk, pk_kind = peaks()
         fine_ms, fine_n = stages["fine"]
@@ -341,6 +360,10 @@ def run_gpu(args, wl):
             "stage_ms": stage_ms,
             "pool_select": {"ms": pool_select_ms, "gbs": qk_bytes / (pool_select_ms / 1e3) / 1e9,
                             "frac_of_hbm": qk_bytes / (pool_select_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+            "reorder": {"ms": reorder_ms, "gbs": reorder_bytes / (reorder_ms / 1e3) / 1e9,
+                        "frac_of_hbm": reorder_bytes / (reorder_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                        "note": "q, k, v to tiled and out back; not part of the forward, which gathers tiles "
+                                "in its loads"},
             "roofline": {"kernel": "fine_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{pk_kind} bf16 burst"},
@@ -359,6 +382,76 @@ def run_gpu(args, wl):
     return 0
 
 
+def run_sweep(args):
+    """The 480p sweep: ms, effective TFLOP/s and density at each (top_p, k_min) point, then the
+    cached-mask steps (lists of step 0 reused on perturbed inputs).  One JSON line."""
+    import torch
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+    from block_sparse_spatiotemporal_b200.inputs import perturb_steps, sweep_points
+
+    wl = WORKLOADS["wan480p_sweep"]
+    dev = torch.device("cuda", 0)
+    q, k, v, masters = make_inputs(wl, keep_f32_masters=True)
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
+    shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16)
+    ws = F.workspace(shape, device=dev)
+    cache, counts, _ = F.new_cache(shape, device=dev)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    points = []
+    for top_p, k_min in sweep_points():
+        def step():
+            F.forward(shape, qd, kd, vd, ws, top_p, k_min, cache=cache, out=out, lse=lse)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        pairs = int(counts.sum().item())
+        F.profile_read()
+        F.profile_enable(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        F.profile_enable(False)
+        stages = F.profile_read()
+        if F.device_status(ws) != 0:
+            raise RuntimeError("device status set in the sweep")
+        ms = e0.elapsed_time(e1) / args.steps
+        fine = stages["fine"][0] / max(stages["fine"][1], 1)
+        flops = pairs * pair_flops(wl.head_dim)
+        points.append({"top_p": top_p, "k_min": k_min, "ms": ms, "fine_ms": fine,
+                       "tflops": flops / (ms / 1e3) / 1e12, "fine_tflops": flops / (fine / 1e3) / 1e12,
+                       "density": pairs / (wl.heads * wl.num_tiles ** 2)})
+    # cached-mask steps: fill the cache on step 0, then reuse it on the perturbed inputs
+    F.forward(shape, qd, kd, vd, ws, wl.top_p, wl.k_min, cache=cache, out=out, lse=lse)
+    torch.cuda.synchronize(dev)
+    pairs = int(counts.sum().item())
+    cached = []
+    for qt, kt in perturb_steps(wl, masters):
+        qx, kx = as_dev(qt), as_dev(kt)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            F.forward(shape, qx, kx, vd, ws, wl.top_p, wl.k_min, cache=cache, reuse_mask=True, out=out, lse=lse)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        cached.append(e0.elapsed_time(e1) / args.steps)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set in the cached steps")
+    line = {"metric": METRIC, "unit": UNIT, "workload": wl.name, "steps": args.steps, "warmup": args.warmup,
+            "sweep": points,
+            "cached_mask": {"top_p": wl.top_p, "k_min": wl.k_min,
+                            "density": pairs / (wl.heads * wl.num_tiles ** 2), "ms_per_step": cached,
+                            "tflops_mean": pairs * pair_flops(wl.head_dim) / (statistics.mean(cached) / 1e3) / 1e12}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -368,11 +461,14 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="wan480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="the 480p top-p / top-k / cached-mask sweep (one JSON line)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)
