@@ -19,7 +19,9 @@ Sources (page title, section):
   * "FVAttn" digest (iselia-ai.com), sections 00 and 02: the routing front end
     is top-p routing with a top-k safety floor.
   * "DFSAttn" digest (gist.science 2605.23445), section 1 "Hilbert shuffle":
-    tokens are reordered along a 3D Hilbert curve before blocking; section 3
+    tokens are reordered along a 3D Hilbert curve before blocking; section 2
+    "sub-block scores": a block is split into smaller sub-blocks, each scored,
+    and the fine scores are summed into the block's importance; section 3
     "smart cache": the previous step's selection is reused.
   * "Causal-RoPE SP" digest (gist.science 2603.06664), sections 2.2-2.3: 3D
     rotary position encoding with precomputed frequencies.
@@ -41,7 +43,15 @@ Readings where the pages are silent (each also listed in the design notes):
     (the tensor-core operand precision of a bf16 workload);
   * Hilbert order: Skilling's transposed-axes Hilbert index ("Programming the
     Hilbert curve", AIP Conf. Proc. 707, 2004) on the enclosing 2^k cube with
-    axes (t, h, w), valid tokens ordered by index.
+    axes (t, h, w), valid tokens ordered by index;
+  * sub-block scoring: a 4x4x4 tile is split into the eight 2x2x2 sub-cubes of
+    its grid coordinates; Q and K are pooled per sub-cube; every query
+    sub-block takes a softmax over all key sub-blocks of the head; the
+    importance of key tile j for query tile i is the mean, over the eight
+    query sub-blocks of i, of the probability mass they give to the eight
+    key sub-blocks of j (the sum of the fine scores, normalised so that each
+    row sums to one); top-p and k_min then act on these tile probabilities,
+    ranked by their logarithm (no underflow ties).
 
 Every function below is pinned by ``tests/test_oracle_*.py`` against brute
 force, closed forms, invariants or library routines; see the pin list in the
@@ -269,6 +279,79 @@ def select_blocks(S, top_p, k_min):
     for r in range(P.shape[0]):
         idx[r, :counts[r]] = np.sort(order[r, :counts[r]])
     return counts, idx, border
+
+
+# ----------------------------------------------------------------------------
+# hierarchical (sub-block) scoring
+# ----------------------------------------------------------------------------
+
+SUB = (2, 2, 2)
+
+
+def subblock_ids(coords_tiled, tile=TILE, sub=SUB):
+    """Sub-block of every tiled row (0 .. S-1, S = tile/sub per axis product),
+    from the token's grid coordinates: raster order of the sub-cube inside its
+    tile.  coords_tiled [N, 3] are the (t, h, w) of the tiled rows."""
+    per = [t // s for t, s in zip(tile, sub)]
+    c = (np.asarray(coords_tiled) % np.array(tile)) // np.array(sub)
+    return (c[:, 0] * per[1] + c[:, 1]) * per[2] + c[:, 2]
+
+
+def pool_subblocks(x_tiled, coords_tiled, tile=TILE, sub=SUB):
+    """Mean of each sub-block of each tile: [N, d] -> [nT, S, d]."""
+    tsz = tile[0] * tile[1] * tile[2]
+    nsub = tsz // (sub[0] * sub[1] * sub[2])
+    N, d = x_tiled.shape
+    nT = N // tsz
+    ids = subblock_ids(coords_tiled, tile, sub)
+    x = np.asarray(x_tiled, np.float64)
+    out = np.zeros((nT, nsub, d))
+    cnt = np.zeros((nT, nsub))
+    tiles = np.arange(N) // tsz
+    np.add.at(out, (tiles, ids), x)
+    np.add.at(cnt, (tiles, ids), 1.0)
+    return out / cnt[:, :, None]
+
+
+def _logsumexp(a, axis):
+    m = np.max(a, axis=axis, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    return np.squeeze(m, axis=axis) + np.log(np.sum(np.exp(a - m), axis=axis))
+
+
+def subblock_tile_logprob(qs, ks, scale):
+    """Tile log-probabilities from sub-block scores: qs [nT, S, d], ks [nT, S, d]
+    -> logP [nT, nT] with P[i, j] = (1/S) sum_a sum_b softmax_{(j', b')}(scale *
+    qs[i, a] . ks[j', b'])[j, b], evaluated in the log domain."""
+    nT, S, d = qs.shape
+    L = scale * (qs.reshape(nT * S, d) @ ks.reshape(nT * S, d).T)       # [(i,a), (j,b)]
+    L = L.reshape(nT, S, nT, S)
+    T = _logsumexp(L, axis=3)                                           # [i, a, j]: mass of key tile j
+    Z = _logsumexp(T, axis=2)                                           # [i, a]: row normaliser
+    return _logsumexp(T - Z[:, :, None], axis=1) - math.log(S)          # [i, j]
+
+
+def coarse_head_subblock(q, k, grid, order, top_p, k_min, scale, rope=None, pos=None, sub=SUB):
+    """Steps 1-4 for one head with sub-block scoring; q, k [N, d] float64 in
+    natural order.  Returns the tile log-probabilities (the ranking key),
+    counts, idx, borderline flags and a per-row magnitude of the sub-block
+    logits' terms (for the float32 near-tie bound)."""
+    if pos is None:
+        pos = positions(grid, order)
+    coords = token_coords(grid)
+    if rope is not None:
+        q = rope_3d(q, coords, rope["dims"], rope["base"])
+        k = rope_3d(k, coords, rope["dims"], rope["base"])
+    qt, kt = to_tiled(q, pos), to_tiled(k, pos)
+    ct = to_tiled(coords, pos)
+    qs, ks = pool_subblocks(qt, ct, sub=sub), pool_subblocks(kt, ct, sub=sub)
+    logP = subblock_tile_logprob(qs, ks, scale)
+    counts, idx, border = select_blocks(logP, top_p, k_min)
+    nT, S, d = qs.shape
+    s_abs = scale * (np.abs(qs.reshape(nT * S, d)) @ np.abs(ks.reshape(nT * S, d)).T)
+    s_abs = s_abs.reshape(nT, S, nT, S).max(axis=(1, 2, 3))
+    return dict(logP=logP, P=np.exp(logP), counts=counts, idx=idx, border=border,
+                qs=qs, ks=ks, s_abs_row=s_abs, pos=pos)
 
 
 def near_tie_rows(S, counts, tol):
