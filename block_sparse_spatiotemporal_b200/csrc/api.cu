@@ -77,7 +77,8 @@ int check_rope(const fvattn_rope* r, const Geom& g) {
   return FVATTN_OK;
 }
 
-WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r) {
+// sub: also the sub-block scoring buffers (pooled sub-blocks, key-tile masses).
+WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = false) {
   WsLayout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -107,6 +108,14 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r) {
   const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
   L.qrot = take(rot);
   L.krot = take(rot);
+  if (sub) {
+    const size_t sb = sizeof(float) * (size_t)g.BH * g.nT * kSubBlocks * g.d;
+    L.sqh = take(sb);
+    L.sql = take(sb);
+    L.skh = take(sb);
+    L.skl = take(sb);
+    L.tmass = take(sizeof(float) * (size_t)g.BH * g.nT * kSubBlocks * g.nT);
+  }
   L.total = off;
   return L;
 }
@@ -179,15 +188,17 @@ int make_tile_map(CUtensorMap* map, const void* base, const Geom& g, bool natura
   return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
-// TMA descriptor over a pooled fp32 [BH, nT, d] tensor (tf32 operand of the
-// score kernel): 3D (d, nT, BH), box = 32 dims (128 bytes) x 128 tiles,
-// 128-byte swizzle; tiles past nT read as zero.
-int make_pooled_map(CUtensorMap* map, const float* base, const Geom& g) {
+// TMA descriptor over a pooled fp32 [BH, rows, d] tensor (tf32 operand of the
+// score kernel; rows = nT tiles, or nT * 8 sub-blocks): 3D (d, rows, BH),
+// box = 32 dims (128 bytes) x 128 rows, 128-byte swizzle; rows past the end
+// read as zero.
+int make_pooled_map(CUtensorMap* map, const float* base, const Geom& g, int rows = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FVATTN_ERR_CUDA;
+  if (rows <= 0) rows = g.nT;
   const cuuint64_t row = (cuuint64_t)g.d * 4;
-  const cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.nT, (cuuint64_t)g.BH};
-  const cuuint64_t strides[2] = {row, row * (cuuint64_t)g.nT};
+  const cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)rows, (cuuint64_t)g.BH};
+  const cuuint64_t strides[2] = {row, row * (cuuint64_t)rows};
   const cuuint32_t box[3] = {32, 128, 1};
   const cuuint32_t es[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
@@ -263,11 +274,11 @@ struct Call {
 };
 
 int begin(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws, size_t ws_bytes,
-          fvattn_stream_t stream) {
+          fvattn_stream_t stream, bool sub = false) {
   FV_TRY(make_geom(shape, &c->g));
   FV_TRY(check_rope(rope, c->g));
   if (!ws || !aligned(ws, kAlign)) return FVATTN_ERR_INVALID_ARG;
-  c->L = layout_for(c->g, shape->dtype, rope);
+  c->L = layout_for(c->g, shape->dtype, rope, sub);
   if (ws_bytes < c->L.total) return FVATTN_ERR_WORKSPACE;
   FV_TRY(device_info(&c->dev));
   c->ws = static_cast<char*>(ws);
@@ -441,6 +452,53 @@ int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k, 
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
   FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, false, top_p, k_min, out));
+  return FVATTN_OK;
+}
+
+int fvattn_workspace_size_subblock(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes) {
+  if (!bytes) return FVATTN_ERR_INVALID_ARG;
+  Geom g{};
+  FV_TRY(make_geom(shape, &g));
+  FV_TRY(check_rope(rope, g));
+  *bytes = layout_for(g, shape->dtype, rope, true).total;
+  return FVATTN_OK;
+}
+
+int fvattn_pool_select_subblock(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
+                                float top_p, int32_t k_min, const fvattn_blocks* out, void* ws, size_t ws_bytes,
+                                fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k)) return FVATTN_ERR_INVALID_ARG;
+  if (std::isnan(top_p) || k_min < 0) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream, true));
+  FV_TRY(check_blocks(out, c.g));
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, !natural));
+  const bool r = rope_on(rope);
+  PooledOut po{};
+  po.hi[0] = c.at<float>(c.L.sqh);
+  po.lo[0] = c.at<float>(c.L.sql);
+  po.hi[1] = c.at<float>(c.L.skh);
+  po.lo[1] = c.at<float>(c.L.skl);
+  {
+    StageTimer t(FVATTN_STAGE_POOL, c.s);
+    FV_CUDA(launch_pool_sub(c.g, shape->dtype, q, k, natural ? 1 : 0, c.at<int>(c.L.tile_cube),
+                            c.at<int>(c.L.tile_tok), r ? 1 : 0, r ? rope->dt : 0, r ? rope->dh : 0, r ? rope->dw : 0,
+                            c.at<float2>(c.L.rope_tab), po, c.s));
+    t.kernels = 1;
+  }
+  StageTimer t(FVATTN_STAGE_SELECT, c.s);
+  const int rows = c.g.nT * kSubBlocks;
+  CUtensorMap mqh, mql, mkh, mkl;
+  FV_TRY(make_pooled_map(&mqh, po.hi[0], c.g, rows));
+  FV_TRY(make_pooled_map(&mql, po.lo[0], c.g, rows));
+  FV_TRY(make_pooled_map(&mkh, po.hi[1], c.g, rows));
+  FV_TRY(make_pooled_map(&mkl, po.lo[1], c.g, rows));
+  ScoreArgs sa{c.g, c.at<float>(c.L.tmass), c.status, kDefaultWaitCap};
+  FV_CUDA(launch_scores_sub(mqh, mql, mkh, mkl, sa, c.s));
+  FV_CUDA(launch_subblock_agg(c.g, sa.S, c.at<float>(c.L.scores), c.s));
+  FV_CUDA(launch_select(c.g, c.at<float>(c.L.scores), top_p, k_min, out->counts, out->idx, out->cap, c.s));
+  t.kernels = 3;
   return FVATTN_OK;
 }
 

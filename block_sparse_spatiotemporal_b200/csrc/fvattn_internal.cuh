@@ -16,6 +16,7 @@ namespace fvattn {
 
 constexpr int kTileTokens = 64;
 constexpr int kItemTiles = 2;   // query tiles per fine-stage work item (one 128-row tile)
+constexpr int kSubBlocks = 8;   // 2x2x2 sub-cubes of a tile in sub-block scoring
 constexpr int kMaxTiles = 8192;
 
 // Device status codes (workspace status word).
@@ -55,6 +56,9 @@ struct WsLayout {
   size_t worklist;       // int32 [BH*P]
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
+  size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
+  size_t skh, skl;       //   ... of K
+  size_t tmass;          //   float [BH*nT*8*nT] log2 key-tile masses per query sub-block
   size_t total;
 };
 
@@ -331,6 +335,12 @@ cudaError_t launch_scores(const CUtensorMap& mqh, const CUtensorMap& mql, const 
                           const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s);
 cudaError_t launch_select(const Geom& g, const float* S, float top_p, int k_min, int* counts, int* idx, int cap,
                           cudaStream_t s);
+cudaError_t launch_pool_sub(const Geom& g, int dtype, const void* q, const void* k, int natural, const int* tile_cube,
+                            const int* tile_tok, int rope_enabled, int dt, int dh, int dw, const float2* rope_tab,
+                            const PooledOut& po, cudaStream_t s);
+cudaError_t launch_scores_sub(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                              const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s);
+cudaError_t launch_subblock_agg(const Geom& g, const float* Tb, float* logp, cudaStream_t s);
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
                          cudaStream_t s);
 cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s);

@@ -9,11 +9,18 @@
 // dropped lo.lo term is below 2^-22 |q||k| per dimension.  The result has
 // about the accuracy of an fp32 FFMA dot product.
 //
-// One CTA per (128 query tiles, head), 192 threads: warp 0 loads the CTA's
-// Qp rows once and streams Kp in 32-dim slices of 128 key tiles (TMA, 3-stage
-// ring); warp 1 issues the MMAs (M=128, N=128, K=8) into one of two TMEM
-// accumulators; warps 2-5 drain a finished 128 x 128 block (thread r = query
-// tile r) to the fp32 score buffer while the next block is computed.
+// One CTA per (128 query rows, head), 192 threads: warp 0 loads the CTA's
+// pooled query rows once and streams pooled key rows in 32-dim slices of 128
+// rows (TMA, 3-stage ring); warp 1 issues the MMAs (M=128, N=128, K=8) into
+// one of two TMEM accumulators; warps 2-5 drain a finished 128 x 128 block
+// (thread r = query row r) while the next block is computed.
+//
+// Two epilogues.  Tile scores (rows = tiles): the scaled logits go to the
+// fp32 score buffer.  Sub-block scores ("DFSAttn" digest, section 2; rows =
+// 2x2x2 sub-blocks, 8 per tile, key sub-blocks of a tile adjacent): every
+// group of 8 columns is one key tile, reduced to T = log2 sum 2^(s log2 e),
+// the log of the unnormalised softmax mass the query sub-block gives that
+// key tile.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
@@ -48,6 +55,18 @@ __device__ inline void mma_tf32_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bde
       : "memory");
 }
 
+__device__ inline float sc_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ inline float sc_lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <bool SUB>
 __global__ void __launch_bounds__(sc::THREADS, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap mqh, const __grid_constant__ CUtensorMap mql,
                     const __grid_constant__ CUtensorMap mkh, const __grid_constant__ CUtensorMap mkl,
@@ -63,7 +82,8 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rb = blockIdx.x, bh = blockIdx.y;
-  const int nkc = (g.nT + 127) / 128;
+  const int rows = SUB ? g.nT * kSubBlocks : g.nT;   // pooled rows per head (query and key alike)
+  const int nkc = (rows + 127) / 128;
   const long long cap = a.wait_cap;
 
   if (threadIdx.x == 0) {
@@ -158,7 +178,8 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
     const int row = 32 * q4 + lane;
     const int grow = rb * 128 + row;
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    float* srow = a.S + ((size_t)bh * g.nT + (grow < g.nT ? grow : 0)) * g.nT;
+    float* srow = a.S + ((size_t)bh * rows + (grow < rows ? grow : 0)) * g.nT;
+    const float sl2 = g.scale * 1.4426950408889634f;
     for (int j = 0; j < nkc; ++j) {
       const int b = j & 1;
       if (!mbar_wait(&ctl.s_full[b], (uint32_t)(j >> 1) & 1, abort_flag, a.status, cap)) break;
@@ -169,7 +190,30 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
         tmem_ld32(tbase + 128 * b + 32 * ch + lane_off, v);
         tmem_wait_ld();
         const int col0 = j * 128 + 32 * ch;
-        if (grow < g.nT) {
+        if (SUB) {
+          // four key tiles of 8 sub-block columns each; tiles past nT are padding
+          if (grow < rows) {
+            float t4[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              float m = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) m = fmaxf(m, __uint_as_float(v[8 * t + i]) * sl2);
+              float z = 0.f;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) z += sc_ex2(fmaf(__uint_as_float(v[8 * t + i]), sl2, -m));
+              t4[t] = m + sc_lg2(z);
+            }
+            const int key_tile0 = col0 / kSubBlocks;
+            if (key_tile0 + 4 <= g.nT && (g.nT & 3) == 0) {
+              *reinterpret_cast<float4*>(srow + key_tile0) = make_float4(t4[0], t4[1], t4[2], t4[3]);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                if (key_tile0 + t < g.nT) srow[key_tile0 + t] = t4[t];
+            }
+          }
+        } else if (grow < g.nT) {
           if (col0 + 32 <= g.nT && (g.nT & 3) == 0) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -195,15 +239,28 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
   }
 }
 
-cudaError_t launch_scores(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
-                          const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s) {
+template <bool SUB>
+static cudaError_t launch_scores_t(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                                   const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s) {
   const int DC = a.g.d / 32;
   const size_t smem = 1024 + (size_t)(2 * DC + 2 * sc::STAGES) * sc::BOX;
-  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(score_tc_kernel<SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.g.nT + 127) / 128, a.g.BH);
-  score_tc_kernel<<<grid, sc::THREADS, smem, s>>>(mqh, mql, mkh, mkl, a);
+  const int rows = SUB ? a.g.nT * kSubBlocks : a.g.nT;
+  dim3 grid((rows + 127) / 128, a.g.BH);
+  score_tc_kernel<SUB><<<grid, sc::THREADS, smem, s>>>(mqh, mql, mkh, mkl, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                          const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s) {
+  return launch_scores_t<false>(mqh, mql, mkh, mkl, a, s);
+}
+
+cudaError_t launch_scores_sub(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mkh,
+                              const CUtensorMap& mkl, const ScoreArgs& a, cudaStream_t s) {
+  return launch_scores_t<true>(mqh, mql, mkh, mkl, a, s);
 }
 
 }  // namespace fvattn

@@ -18,7 +18,8 @@ import torch
 __all__ = [
     "FvattnError", "Shape", "Rope", "Blocks", "MaskCache", "lib", "library_path",
     "F32", "BF16", "RASTER_CUBE", "HILBERT", "NATURAL", "TILED",
-    "make_shape", "make_rope", "num_tiles", "workspace_size", "workspace",
+    "make_shape", "make_rope", "num_tiles", "workspace_size", "workspace", "workspace_size_subblock",
+    "pool_select_subblock",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
     "STAGES", "pool_select_noalloc",
@@ -80,6 +81,10 @@ _SIGS = {
     "fvattn_pool_select": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
                            ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p,
                            ctypes.c_size_t, ctypes.c_void_p],
+    "fvattn_workspace_size_subblock": [ctypes.POINTER(Shape), ctypes.POINTER(Rope), ctypes.POINTER(ctypes.c_size_t)],
+    "fvattn_pool_select_subblock": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
+                                    ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p,
+                                    ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_pool_select_noalloc": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
                                    ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p],
     "fvattn_build_worklist": [ctypes.POINTER(Shape), ctypes.POINTER(Blocks), ctypes.c_void_p, ctypes.c_void_p,
@@ -162,9 +167,18 @@ def workspace_size(shape: Shape, rope: Optional[Rope] = None) -> int:
     return n.value
 
 
-def workspace(shape: Shape, rope: Optional[Rope] = None, device="cuda") -> torch.Tensor:
-    """A device workspace of the size the library asks for (caller-owned)."""
-    return torch.empty(workspace_size(shape, rope), dtype=torch.uint8, device=device)
+def workspace(shape: Shape, rope: Optional[Rope] = None, device="cuda", subblock=False) -> torch.Tensor:
+    """A device workspace of the size the library asks for (caller-owned);
+    ``subblock`` sizes it for pool_select_subblock as well."""
+    n = workspace_size_subblock(shape, rope) if subblock else workspace_size(shape, rope)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def workspace_size_subblock(shape: Shape, rope: Optional[Rope] = None) -> int:
+    n = ctypes.c_size_t()
+    _check("fvattn_workspace_size_subblock",
+           lib().fvattn_workspace_size_subblock(ctypes.byref(shape), _rope_ptr(rope), ctypes.byref(n)))
+    return n.value
 
 
 def new_blocks(shape: Shape, device="cuda"):
@@ -204,6 +218,20 @@ def pool_select(shape: Shape, q, k, ws, top_p: float, k_min: int, rope: Optional
     _check("fvattn_pool_select", lib().fvattn_pool_select(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope),
                                                           float(top_p), int(k_min), ctypes.byref(b), _ptr(ws),
                                                           ws.numel(), _stream(stream)))
+    return counts, idx
+
+
+def pool_select_subblock(shape: Shape, q, k, ws, top_p: float, k_min: int, rope: Optional[Rope] = None,
+                         blocks=None, stream=None):
+    """Steps 2-5 with hierarchical sub-block scoring (ws from
+    ``workspace(..., subblock=True)``): returns (counts, idx)."""
+    if blocks is None:
+        counts, idx, b = new_blocks(shape, q.device)
+    else:
+        counts, idx, b = blocks
+    _check("fvattn_pool_select_subblock",
+           lib().fvattn_pool_select_subblock(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope), float(top_p),
+                                             int(k_min), ctypes.byref(b), _ptr(ws), ws.numel(), _stream(stream)))
     return counts, idx
 
 

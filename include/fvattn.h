@@ -134,6 +134,25 @@ int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k,
                        const fvattn_blocks* out, void* ws, size_t ws_bytes,
                        fvattn_stream_t stream);
 
+/* Steps 2-5 with hierarchical sub-block scoring ("DFSAttn" digest, section 2:
+ * a block is split into smaller sub-blocks whose scores are summed into the
+ * block's importance).  Each 4x4x4 tile splits into the eight 2x2x2
+ * sub-cubes of its grid coordinates; Q and K are mean-pooled per sub-cube;
+ * every query sub-block takes a softmax over all key sub-blocks of the
+ * head; the importance of key tile j for query tile i is the mean over the
+ * eight query sub-blocks of i of the probability mass they give to the
+ * eight key sub-blocks of j.  Top-p and k_min act on these importances
+ * exactly as in fvattn_pool_select (ranked by their logarithm, ties to the
+ * lower tile id).  Arguments, layouts and results as fvattn_pool_select;
+ * the workspace is fvattn_workspace_size_subblock bytes (it adds
+ * 4 * B*H*nT*8*d + B*H*nT*8*nT floats).  The fine stage for these lists is
+ * fvattn_block_sparse_fwd. */
+int fvattn_workspace_size_subblock(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes);
+int fvattn_pool_select_subblock(const fvattn_shape* shape, const void* q, const void* k,
+                                const fvattn_rope* rope, float top_p, int32_t k_min,
+                                const fvattn_blocks* out, void* ws, size_t ws_bytes,
+                                fvattn_stream_t stream);
+
 /* Steps 2-5 without a caller workspace.  The pages have no counterpart:
  * this is for callers that cannot allocate device memory (a plugin whose
  * host application owns every device allocation and passes in only the
