@@ -232,14 +232,18 @@ def run_gpu(args, wl):
     shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16,
                          order=F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE)
     rope = F.make_rope(wl.rope_dims, wl.rope_base) if wl.rope else None
-    ws = F.workspace(shape, rope, device=dev)
-    cache, counts, _ = F.new_cache(shape, device=dev)
+    ws = F.workspace(shape, rope, device=dev, subblock=args.subblock)
+    cache, counts, idx = F.new_cache(shape, device=dev)
     out = torch.empty_like(qd)
     lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(qx=qd, kx=kd, vx=vd):
-        F.forward(shape, qx, kx, vx, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=out, lse=lse)
+        if args.subblock:   # sub-block scoring, then the fine stage on its lists
+            F.pool_select_subblock(shape, qx, kx, ws, wl.top_p, wl.k_min, rope=rope, blocks=(counts, idx, cache.blocks))
+            F.block_sparse_fwd(shape, qx, kx, vx, counts, idx, ws, rope=rope, out=out, lse=lse)
+        else:
+            F.forward(shape, qx, kx, vx, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=out, lse=lse)
 
     for _ in range(max(args.warmup, 1)):
         step()
@@ -354,6 +358,7 @@ def run_gpu(args, wl):
             "config": {"workload": wl.name, "grid": list(wl.grid), "tokens": wl.tokens, "heads": wl.heads,
                        "head_dim": wl.head_dim, "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order,
                        "rope": wl.rope, "selected_pairs": pairs,
+                       "scoring": "sub-block 2x2x2" if args.subblock else "tile mean",
                        "density": pairs / (wl.heads * wl.num_tiles ** 2),
                        "l2": "inputs larger than L2 (q+k+v = %.0f MB)" % (3 * qk_bytes / 2 / 1e6),
                        "parallelism": f"replica x{world}"},
@@ -462,6 +467,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="the 480p top-p / top-k / cached-mask sweep (one JSON line)")
+    ap.add_argument("--subblock", action="store_true",
+                    help="hierarchical sub-block scoring (pool_select_subblock + block_sparse_fwd)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

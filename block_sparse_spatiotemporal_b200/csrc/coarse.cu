@@ -41,65 +41,6 @@ __global__ void rope_table_kernel(Geom g, int dt, int dh, int dw, float base, fl
   }
 }
 
-// Vector load / store of DPL consecutive elements as fp32.
-template <typename T, int DPL> struct Vec;
-template <int DPL> struct Vec<float, DPL> {
-  static __device__ inline void load(const float* p, float (&v)[DPL]) {
-    if constexpr (DPL == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(p);
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else if constexpr (DPL == 2) {
-      const float2 t = *reinterpret_cast<const float2*>(p);
-      v[0] = t.x; v[1] = t.y;
-    } else {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) v[i] = p[i];
-    }
-  }
-  static __device__ inline void store(float* p, const float (&v)[DPL]) {
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    } else if constexpr (DPL == 2) {
-      *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) p[i] = v[i];
-    }
-  }
-};
-template <int DPL> struct Vec<__nv_bfloat16, DPL> {
-  static_assert(DPL % 2 == 0, "bf16 rows are read in pairs");
-  static __device__ inline void load(const __nv_bfloat16* p, float (&v)[DPL]) {
-    uint32_t w[DPL / 2];
-    if constexpr (DPL == 4) {
-      const uint2 t = *reinterpret_cast<const uint2*>(p);
-      w[0] = t.x; w[1] = t.y;
-    } else {
-#pragma unroll
-      for (int i = 0; i < DPL / 2; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
-    }
-#pragma unroll
-    for (int i = 0; i < DPL / 2; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-  static __device__ inline void store(__nv_bfloat16* p, const float (&v)[DPL]) {
-    uint32_t w[DPL / 2];
-#pragma unroll
-    for (int i = 0; i < DPL / 2; ++i) {
-      __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&b);
-    }
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < DPL / 2; ++i) reinterpret_cast<uint32_t*>(p)[i] = w[i];
-    }
-  }
-};
-
 // Rotate the pair (a, b) = dims (dim, dim+1) of a token at (t, h, w).
 __device__ inline void rope_pair(const RopeArgs& r, const Geom& g, int dim, int t, int h, int w, float& a,
                                  float& b) {

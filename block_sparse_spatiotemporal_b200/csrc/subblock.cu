@@ -38,11 +38,6 @@ __device__ inline int sub_of(int t, int h, int w) {
   return (((t & 3) >> 1) << 2) | (((h & 3) >> 1) << 1) | ((w & 3) >> 1);
 }
 
-// Element load of one head-dim slice as fp32.
-template <typename T> __device__ inline float ld_f32(const T* p);
-template <> __device__ inline float ld_f32<float>(const float* p) { return *p; }
-template <> __device__ inline float ld_f32<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-
 // One block per (tile, head, tensor), 128 threads.  Warp w reads rows w,
 // w + 4, ... of the tile (lanes over head dims) and adds each row into the
 // running sum of its sub-cube; the four warps' partial sums are added in warp
@@ -71,8 +66,7 @@ __global__ void __launch_bounds__(128) pool_sub_kernel(Geom g, const T* __restri
     const int sb = sub_of(t, h, w);
     const T* row = x + ((size_t)bh * g.N + n) * D + lane * DPL;
     float v[DPL];
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) v[i] = ld_f32<T>(row + i);
+    Vec<T, DPL>::load(row, v);
     if (rope.enabled) {
 #pragma unroll
       for (int i = 0; i < DPL; i += 2) {
