@@ -43,7 +43,7 @@ namespace fvattn {
 namespace ft {
 
 #ifndef FVATTN_FT_KSTAGES
-#define FVATTN_FT_KSTAGES 2
+#define FVATTN_FT_KSTAGES 3
 #endif
 #ifndef FVATTN_FT_VSTAGES
 #define FVATTN_FT_VSTAGES 3
@@ -81,12 +81,13 @@ struct Ctl {
                            // c waits for PV(c - 2), and PV(c + 2) needs P(c + 2), so a waiter
                            // never sees two outstanding phases)
   uint64_t o_empty;        // epilogue read both O (256 arrivals per item)
-  uint64_t xchg;           // epilogue (m, l) exchange between the halves (256 per item)
+  uint64_t xchg1;          // epilogue: group 1 published (m, l) (128 arrivals per item)
+  uint64_t xchg2;          // epilogue: group 0 replaced them with the merge scales (128 per item)
   uint64_t drain;          // final commits of the two MMA threads
   int info[SBUF];          // per S buffer: the step word
   int meta[KST];
-  float xm[2][128], xl[2][128];   // epilogue exchange [group][row] (a group rewrites its slot only
-                                  // after the other group's P of the next step, so after its read)
+  float2 ex[128];                 // epilogue exchange per row: group 1's (m, l), then the scales
+                                  // (s0, s1) group 0 computed from both groups' (m, l)
   uint32_t tmem_base;
   int abort;
 };
@@ -299,7 +300,8 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       mbar_init(&ctl->pv_done[i], 1);
     }
     mbar_init(&ctl->o_empty, 256);
-    mbar_init(&ctl->xchg, 256);
+    mbar_init(&ctl->xchg1, 128);
+    mbar_init(&ctl->xchg2, 128);
     mbar_init(&ctl->drain, 2);           // one final commit per MMA thread
     ctl->abort = 0;
     fence_mbar_init();
@@ -593,18 +595,28 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       // ---- epilogue: merge the groups' (m, l, O); this group writes dims 64 h .. 64 h + 63
       if (!mbar_wait(&ctl->pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) break;
       tc_fence_after();
-      ctl->xm[h][r] = m_use;
-      ctl->xl[h][r] = l;
-      mbar_arrive(&ctl->xchg);
-      if (!mbar_wait(&ctl->xchg, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
-      const float m0 = ctl->xm[0][r], m1 = ctl->xm[1][r];
-      const float l0 = ctl->xl[0][r], l1 = ctl->xl[1][r];
-      const float M = fmaxf(m0, m1);
-      const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
-      const float w1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
-      const float L = l0 * w0 + l1 * w1;
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      const float s0 = w0 * inv, s1 = w1 * inv;
+      // group 1 publishes (m, l); group 0 merges and writes back both scales into the same slot
+      float s0 = 0.f, s1 = 0.f, M = -INFINITY, L = 0.f;
+      if (h == 1) {
+        ctl->ex[r] = make_float2(m_use, l);
+        mbar_arrive(&ctl->xchg1);
+        if (!mbar_wait(&ctl->xchg2, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
+        const float2 sc = ctl->ex[r];
+        s0 = sc.x;
+        s1 = sc.y;
+      } else {
+        if (!mbar_wait(&ctl->xchg1, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
+        const float2 o1 = ctl->ex[r];
+        M = fmaxf(m_use, o1.x);
+        const float w0 = m_use == -INFINITY ? 0.f : ex2(m_use - M);
+        const float w1 = o1.x == -INFINITY ? 0.f : ex2(o1.x - M);
+        L = l * w0 + o1.y * w1;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        s0 = w0 * inv;
+        s1 = w1 * inv;
+        ctl->ex[r] = make_float2(s0, s1);
+        mbar_arrive(&ctl->xchg2);
+      }
       const int tok = !valid ? 0 : (a.out_nat ? cube_row_token(g, cube, rr) : tile * kTileTokens + rr);
       __nv_bfloat16* orow = a.out + ((size_t)bh * g.N + tok) * D + 64 * h;
       const uint32_t tO0 = tbase + TMEM_O + lane_off + 64 * h, tO1 = tO0 + 128;
