@@ -39,6 +39,14 @@ rounded to bf16 on its own.
 
 Token layout: natural order is raster order over the latent grid (T, Hg, W),
 index n = (t * Hg + h) * W + w, tensors are [B, H, N, d] with B = 1.
+
+Prologue inputs (the QKV projection before attention): token features
+X [B, N, C] ~ N(0, 1) (the scale of normalised DiT activations), weights
+W [3*H*d, C] ~ N(0, 1/C) (fan-in initialisation, so projected values are
+about N(0, 1)) and bias [3*H*d] ~ N(0, 0.1^2), all rounded to bf16 except the
+float32 bias.  X rows are drawn in chunks of 4096 tokens, chunk c of batch b
+from ``default_rng(SeedSequence([seed, 200, b, c]))``; W and bias from
+``default_rng(SeedSequence([seed, 201]))`` and ``[seed, 202]``.
 """
 from __future__ import annotations
 
@@ -48,7 +56,8 @@ import math
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "perturb_steps",
-           "f32_to_bf16_bits", "bf16_bits_to_f32", "sweep_points"]
+           "f32_to_bf16_bits", "bf16_bits_to_f32", "sweep_points",
+           "make_projection_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -227,3 +236,23 @@ def perturb_steps(wl: Workload, masters: dict, steps: int = 10):
             km[b, h] += np.float32(0.05) * _noise([wl.seed, 100 + t, 1, b, h], (N, d))
         _parallel(one, [(b, h) for b in range(B) for h in range(H)])
         yield _finish(qm, wl), _finish(km, wl)
+
+
+def make_projection_inputs(batch: int, tokens: int, channels: int, heads: int, head_dim: int,
+                           seed: int, bias: bool = True):
+    """Draw (x, w, b) for the QKV projection: x [B, N, C] and w [3*H*d, C] as
+    bf16 bit patterns (uint16), b [3*H*d] float32 or None."""
+    chunk = 4096
+    x = np.empty((batch, tokens, channels), np.uint16)
+
+    def one(item):
+        b, c = item
+        lo, hi = c * chunk, min(tokens, (c + 1) * chunk)
+        x[b, lo:hi] = f32_to_bf16_bits(_noise([seed, 200, b, c], (hi - lo, channels)))
+
+    _parallel(one, [(b, c) for b in range(batch) for c in range((tokens + chunk - 1) // chunk)])
+    rows = 3 * heads * head_dim
+    w32 = _noise([seed, 201], (rows, channels)) * np.float32(1.0 / math.sqrt(channels))
+    w = f32_to_bf16_bits(w32)
+    bv = (_noise([seed, 202], (rows,)) * np.float32(0.1)).astype(np.float32) if bias else None
+    return x, w, bv

@@ -51,7 +51,12 @@ Readings where the pages are silent (each also listed in the design notes):
     query sub-blocks of i, of the probability mass they give to the eight
     key sub-blocks of j (the sum of the fine scores, normalised so that each
     row sums to one); top-p and k_min then act on these tile probabilities,
-    ranked by their logarithm (no underflow ties).
+    ranked by their logarithm (no underflow ties);
+  * prologue: Q | K | V = X W^T + b, one linear layer whose 3*H*d output
+    rows are Q heads, then K heads, then V heads (head h of each at rows
+    h*d..h*d+d-1); Q and K are rotated by the 3D RoPE above at
+    (t + s, h, w), s the start frame of the block ("Causal-RoPE SP" digest,
+    section 2.2), V is not; the results are rounded once to bf16.
 
 Every function below is pinned by ``tests/test_oracle_*.py`` against brute
 force, closed forms, invariants or library routines; see the pin list in the
@@ -215,6 +220,83 @@ def round_bf16(x):
     scaled = np.ldexp(m, 8)                # 8 significant bits
     r = np.round(scaled)                   # numpy rounds half to even
     return np.ldexp(r, e - 8)
+
+
+# ----------------------------------------------------------------------------
+# prologue: QKV projection fused with the 3D rotary encoding
+# ----------------------------------------------------------------------------
+
+def project_qkv(x, w, bias=None):
+    """Linear projection of token features to Q | K | V columns.
+
+    x [..., C] float64, w [3*H*d, C] float64 (output rows first, as a linear
+    layer stores them), bias [3*H*d] or None.  Returns x @ w^T + bias."""
+    y = np.asarray(x, np.float64) @ np.asarray(w, np.float64).T
+    if bias is not None:
+        y = y + np.asarray(bias, np.float64)
+    return y
+
+
+def qkv_rope(x, w, bias, grid, heads, head_dim, rope=None, t_offset=0,
+             order=None, tokens=None, rounded=True):
+    """The attention prologue ("Causal-RoPE SP" digest, section 2.3: QKV
+    projection and the rotary encoding as one operator; section 2.2: a token
+    at local frame t of a block that starts at frame s is encoded at global
+    frame t + s).
+
+    x [B, N, C] float64 in natural token order; w [3*H*d, C]; bias or None.
+    Output columns o = which*H*d + h*d + j: which 0/1/2 = Q/K/V, head h,
+    head dim j.  Q and K of token n are rotated by ``rope_3d`` at
+    (t + t_offset, h, w); V is not rotated.  ``rounded`` rounds the results
+    once to bf16.  Returns q, k, v [B, H, N, d] in natural order, or in the
+    tiled order ``order`` ("raster" / "hilbert") when given.  ``tokens``
+    (natural indices) restricts the result to those tokens, returned as
+    [B, H, len(tokens), d] in the given order (``order`` must then be None)."""
+    x = np.asarray(x, np.float64)
+    B, N, _ = x.shape
+    H, d = heads, head_dim
+    if tokens is None:
+        tok = np.arange(N)
+    else:
+        if order is not None:
+            raise ValueError("tokens and order are exclusive")
+        tok = np.asarray(tokens, np.int64)
+    y = project_qkv(x[:, tok, :], w, bias)                   # [B, n, 3*H*d]
+    y = y.reshape(B, len(tok), 3, H, d).transpose(2, 0, 3, 1, 4)  # [3, B, H, n, d]
+    q, k, v = y[0].copy(), y[1].copy(), y[2].copy()
+    if rope is not None:
+        coords = token_coords(grid)[tok].copy()
+        coords[:, 0] += t_offset
+        for b in range(B):
+            for h in range(H):
+                q[b, h] = rope_3d(q[b, h], coords, rope["dims"], rope["base"])
+                k[b, h] = rope_3d(k[b, h], coords, rope["dims"], rope["base"])
+    if rounded:
+        q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+    if order is not None:
+        pos = positions(grid, order)
+        q, k, v = to_tiled(q, pos), to_tiled(k, pos), to_tiled(v, pos)
+    return q, k, v
+
+
+def qkv_abs_bound(x, w, bias, heads, head_dim, tokens=None):
+    """Sum over the contraction of |x_c * w_oc| (+ |bias_o|) per output, as
+    [3, B, H, n, d]: the scale of the rounding error of any summation order
+    of the projection (RoPE mixes the two members of a pair, so the bound of a
+    rotated pair is the larger of the two)."""
+    x = np.abs(np.asarray(x, np.float64))
+    if tokens is not None:
+        x = x[:, np.asarray(tokens, np.int64), :]
+    y = x @ np.abs(np.asarray(w, np.float64)).T
+    if bias is not None:
+        y = y + np.abs(np.asarray(bias, np.float64))
+    B, n, _ = y.shape
+    y = y.reshape(B, n, 3, heads, head_dim).transpose(2, 0, 3, 1, 4)
+    pair = np.maximum(y[..., 0::2], y[..., 1::2])
+    y = y.copy()
+    y[..., 0::2] = pair
+    y[..., 1::2] = pair
+    return y
 
 
 # ----------------------------------------------------------------------------
