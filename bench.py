@@ -457,6 +457,121 @@ def run_sweep(args):
     return 0
 
 
+def run_prologue(args, wl):
+    """The attention prologue at the workload's shape: X [1, N, C = H*d] and a
+    linear layer W [3*H*d, C] (+ bias) projected to Q, K, V with the 3D RoPE
+    on Q and K, written in the workload's tiled order.  One JSON line; cuBLAS
+    time of the bare X W^T product (no bias, rotation or reorder) beside it."""
+    import torch
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+    from block_sparse_spatiotemporal_b200.inputs import make_projection_inputs
+
+    dev = torch.device("cuda", 0)
+    B, N, H, d = wl.batch, wl.tokens, wl.heads, wl.head_dim
+    C = H * d
+    x, w, b = make_projection_inputs(B, N, C, H, d, wl.seed)
+    xd = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+    bd = torch.from_numpy(b).to(dev)
+    shape = F.make_shape(B, H, d, wl.grid, dtype=F.BF16,
+                         order=F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE, layout=F.TILED)
+    rope = F.make_rope(wl.rope_dims, wl.rope_base)
+    ws = torch.empty(F.workspace_size_qkv(shape, rope), dtype=torch.uint8, device=dev)
+    out = tuple(torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+    flops = 2.0 * B * N * C * 3 * H * d
+
+    def step(xx=xd):
+        F.qkv_rope(shape, xx, wd, ws, bias=bd, rope=rope, t_offset=0, out=out)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+    sampler = ClockSampler([0])
+    sampler.start()
+    time.sleep(0.3)
+    F.profile_read()
+    F.profile_enable(True)
+    ms = timed(step, args.steps)
+    F.profile_enable(False)
+    stages = F.profile_read()
+    clocks = sampler.stop()
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during the timed region")
+    k_ms, k_n = stages["prologue"]
+    kernel_ms = k_ms / max(k_n, 1)
+
+    x2 = xd.view(B * N, C)
+    for _ in range(3):
+        torch.matmul(x2, wd.t())
+    cublas_ms = timed(lambda: torch.matmul(x2, wd.t()), max(3, min(args.steps, 20)))
+
+    # end to end: pinned host X in, q, k, v back to pinned host buffers
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = tuple(torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory() for _ in range(3))
+    xb = torch.empty_like(xd)
+
+    def e2e_step():
+        xb.copy_(xh, non_blocking=True)
+        step(xb)
+        for o, hst in zip(out, oh):
+            hst.copy_(o, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = timed(e2e_step, max(3, min(args.steps, 10)))
+
+    pk, pk_kind = peaks()
+    achieved = flops / (kernel_ms / 1e3) / 1e12
+    line = {
+        "metric": "QKV projection + 3D RoPE prologue ms & TFLOP/s", "value": flops / (ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"prologue_{wl.name}", "grid": list(wl.grid), "tokens": N, "channels": C,
+                   "heads": H, "head_dim": d, "order": wl.order, "rope": list(wl.rope_dims), "bias": True,
+                   "layout": "tiled", "l2": "inputs larger than L2 (X = %.0f MB, W = %.0f MB)"
+                   % (xd.numel() * 2 / 1e6, wd.numel() * 2 / 1e6)},
+        "stage_ms": {k: round(v[0] / args.steps, 4) for k, v in stages.items() if v[1]},
+        "roofline": {"kernel": "qkv_rope_kernel", "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk_kind} bf16 burst"},
+        "cublas_gemm": {"ms": cublas_ms, "tflops": flops / (cublas_ms / 1e3) / 1e12,
+                        "note": "torch.matmul(X, W^T) alone: no bias, rotation or tiled scatter"},
+        "gpu_launches": sum(n for _, n in stages.values()),
+        "clocks": clocks,
+        "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": xh.numel() * 2, "d2h_bytes_per_step": sum(o.numel() * 2 for o in oh)},
+    }
+    if not args.no_cpu_baseline:
+        from oracle import fvattn_oracle as O
+        rng = np.random.default_rng(0)
+        orope = dict(dims=wl.rope_dims, base=wl.rope_base)
+        n_tok, t0 = 0, time.perf_counter()
+        wf, bf = O.as_f64(w, "bf16"), b.astype(np.float64)
+        while time.perf_counter() - t0 < args.cpu_budget / 2 or n_tok == 0:
+            toks = np.sort(rng.choice(N, 64, replace=False))
+            O.qkv_rope(O.as_f64(x[:, toks], "bf16"), wf, bf, wl.grid, H, d, orope, tokens=toks, gathered=True)
+            n_tok += 64
+        el = time.perf_counter() - t0
+        est = el * (B * N) / n_tok
+        line["cpu_baseline"] = {"value": flops / est / 1e12, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                                "sample": f"oracle (numpy fp64) prologue of {n_tok} random tokens, scaled to "
+                                          f"{B * N} tokens", "est_ms_per_step": est * 1e3}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -469,6 +584,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="the 480p top-p / top-k / cached-mask sweep (one JSON line)")
     ap.add_argument("--subblock", action="store_true",
                     help="hierarchical sub-block scoring (pool_select_subblock + block_sparse_fwd)")
+    ap.add_argument("--prologue", action="store_true",
+                    help="the fused QKV projection + 3D RoPE prologue at the workload's shape (one JSON line)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -476,6 +593,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.sweep:
         return run_sweep(args)
+    if args.prologue:
+        return run_prologue(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)

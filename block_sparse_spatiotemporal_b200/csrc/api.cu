@@ -120,6 +120,26 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   return L;
 }
 
+// Prologue workspace: tables only.
+WsLayout layout_qkv(const Geom& g, const fvattn_rope* r) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.tile_cube = take(sizeof(int) * g.nT);
+  L.cube_rank = take(sizeof(int) * g.nT);
+  L.tok_pos = take(sizeof(int) * (size_t)g.N);
+  const size_t rope_pairs =
+      rope_on(r) ? (size_t)g.T * (r->dt / 2) + (size_t)g.Hg * (r->dh / 2) + (size_t)g.W * (r->dw / 2) : 0;
+  L.rope_pairs = take(sizeof(float2) * rope_pairs);
+  L.total = off;
+  return L;
+}
+
 struct DeviceInfo {
   int sms = 0;
   int major = 0;
@@ -207,6 +227,23 @@ int make_pooled_map(CUtensorMap* map, const float* base, const Geom& g, int rows
   return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
 }
 
+// TMA descriptor over a bf16 [rows, cols] row-major matrix (cols a multiple
+// of 64): box = box_k columns (64 -> 128-byte swizzle, 32 -> 64-byte
+// swizzle) x box_rows rows; rows past the end read as zero.
+int make_rows_map(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows, int box_k) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FVATTN_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_k, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Optional per-stage timing with CUDA events (host objects only).
 // ---------------------------------------------------------------------------
@@ -279,6 +316,21 @@ int begin(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws,
   FV_TRY(check_rope(rope, c->g));
   if (!ws || !aligned(ws, kAlign)) return FVATTN_ERR_INVALID_ARG;
   c->L = layout_for(c->g, shape->dtype, rope, sub);
+  if (ws_bytes < c->L.total) return FVATTN_ERR_WORKSPACE;
+  FV_TRY(device_info(&c->dev));
+  c->ws = static_cast<char*>(ws);
+  c->status = c->at<int>(c->L.status);
+  c->s = reinterpret_cast<cudaStream_t>(stream);
+  FV_CUDA(cudaMemsetAsync(c->status, 0, sizeof(int), c->s));
+  return FVATTN_OK;
+}
+
+int begin_qkv(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws, size_t ws_bytes,
+              fvattn_stream_t stream) {
+  FV_TRY(make_geom(shape, &c->g));
+  FV_TRY(check_rope(rope, c->g));
+  if (!ws || !aligned(ws, kAlign)) return FVATTN_ERR_INVALID_ARG;
+  c->L = layout_qkv(c->g, rope);
   if (ws_bytes < c->L.total) return FVATTN_ERR_WORKSPACE;
   FV_TRY(device_info(&c->dev));
   c->ws = static_cast<char*>(ws);
@@ -563,6 +615,84 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
     cache->k_min = k_min;
     cache->valid = 1;
   }
+  return FVATTN_OK;
+}
+
+int fvattn_workspace_size_qkv(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes) {
+  if (!bytes) return FVATTN_ERR_INVALID_ARG;
+  Geom g{};
+  FV_TRY(make_geom(shape, &g));
+  FV_TRY(check_rope(rope, g));
+  *bytes = layout_qkv(g, rope).total;
+  return FVATTN_OK;
+}
+
+#ifndef FVATTN_QKV_VARIANT
+#define FVATTN_QKV_VARIANT 1   // 128 x 256 tiles, double-buffered accumulators
+#endif
+#ifndef FVATTN_QKV_GROUP_M
+#define FVATTN_QKV_GROUP_M 8
+#endif
+
+int fvattn_qkv_rope(const fvattn_shape* shape, const void* x, int32_t channels, const void* w, const float* bias,
+                    const fvattn_rope* rope, int32_t t_offset, void* q, void* k, void* v, void* ws, size_t ws_bytes,
+                    fvattn_stream_t stream) {
+  if (!tensor_ok(x) || !tensor_ok(w) || !tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v))
+    return FVATTN_ERR_INVALID_ARG;
+  if (bias && !aligned(bias, 16)) return FVATTN_ERR_INVALID_ARG;
+  if (t_offset < 0 || t_offset > (1 << 20)) return FVATTN_ERR_INVALID_ARG;
+  if (!shape) return FVATTN_ERR_INVALID_ARG;
+  if (shape->dtype != FVATTN_BF16) return FVATTN_ERR_DTYPE;
+  if (channels < 64 || channels > 65536 || channels % 64) return FVATTN_ERR_SHAPE;
+  Call c;
+  FV_TRY(begin_qkv(&c, shape, rope, ws, ws_bytes, stream));
+  const Geom& g = c.g;
+  const bool tiled = shape->layout == FVATTN_LAYOUT_TILED;
+  const bool r = rope_on(rope);
+  {
+    StageTimer t(FVATTN_STAGE_TABLES, c.s);
+    if (tiled) {
+      FV_CUDA(launch_tile_table(g, c.at<int>(c.L.tile_cube), c.at<int>(c.L.cube_rank), c.s));
+      FV_CUDA(launch_token_pos(g, c.at<int>(c.L.cube_rank), c.at<int>(c.L.tok_pos), c.s));
+      t.kernels += 2;
+    }
+    if (r) {
+      FV_CUDA(launch_rope_pairs(g, rope->dt, rope->dh, rope->dw, rope->base, t_offset, c.at<float2>(c.L.rope_pairs),
+                                c.s));
+      t.kernels += 1;
+    }
+  }
+  const int variant = FVATTN_QKV_VARIANT;
+  const long long M = (long long)g.B * g.N;
+  const int Nout = 3 * g.H * g.d;
+  const QkvTma tm = qkv_tma(variant);
+  CUtensorMap mx, mw;
+  FV_TRY(make_rows_map(&mx, x, M, channels, tm.box_rows, tm.box_k));
+  FV_TRY(make_rows_map(&mw, w, Nout, channels, 256, tm.box_k));
+  QkvArgs a{};
+  a.bias = bias;
+  a.out[0] = static_cast<__nv_bfloat16*>(q);
+  a.out[1] = static_cast<__nv_bfloat16*>(k);
+  a.out[2] = static_cast<__nv_bfloat16*>(v);
+  a.pos = tiled ? c.at<int>(c.L.tok_pos) : nullptr;
+  a.rope_tab = r ? c.at<float2>(c.L.rope_pairs) : nullptr;
+  a.dt = r ? rope->dt : 0;
+  a.dh = r ? rope->dh : 0;
+  a.dw = r ? rope->dw : 0;
+  a.M = (int)M;
+  a.N = g.N;
+  a.H = g.H;
+  a.T = g.T;
+  a.Hg = g.Hg;
+  a.W = g.W;
+  a.Nout = Nout;
+  a.kblocks = channels / tm.box_k;
+  a.group_m = FVATTN_QKV_GROUP_M;
+  a.status = c.status;
+  a.wait_cap = kDefaultWaitCap;
+  StageTimer t(FVATTN_STAGE_PROLOGUE, c.s);
+  FV_CUDA(launch_qkv(mx, mw, a, variant, c.dev.sms, c.s));
+  t.kernels = 1;
   return FVATTN_OK;
 }
 

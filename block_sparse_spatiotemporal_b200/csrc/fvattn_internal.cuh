@@ -59,6 +59,8 @@ struct WsLayout {
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
   size_t skh, skl;       //   ... of K
   size_t tmass;          //   float [BH*nT*8*nT] log2 key-tile masses per query sub-block
+  size_t tok_pos;        // prologue only: int32 [N] tiled row of natural token n
+  size_t rope_pairs;     //   float2 pair-major (cos, sin) table at the start-frame offset
   size_t total;
 };
 
@@ -92,6 +94,22 @@ struct FineTcArgs {
   __nv_bfloat16* out;
   float* lse;
   int out_nat;
+  int* status;
+  long long wait_cap;
+};
+
+// Prologue: Q | K | V = X W^T (+ bias), RoPE on Q and K, bf16 out.
+struct QkvArgs {
+  const float* bias;       // [Nout] or null
+  __nv_bfloat16* out[3];   // q, k, v: [B, H, N, 128]
+  const int* pos;          // [N] output row of natural token n, or null (natural layout)
+  const float2* rope_tab;  // pair-major: [dt/2][T] | [dh/2][Hg] | [dw/2][W] (cos, sin), or null
+  int dt, dh, dw;
+  int M;                   // B * N rows of X
+  int N, H, T, Hg, W;
+  int Nout;                // 3 * H * 128 rows of W
+  int kblocks;             // C / 64
+  int mt, nt, n_tiles, group_m;
   int* status;
   long long wait_cap;
 };
@@ -269,6 +287,14 @@ __device__ inline bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, l
   return false;
 }
 
+__device__ inline void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 __device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                    int c2) {
   asm volatile(
@@ -368,6 +394,17 @@ __device__ inline uint64_t umma_desc_sw128(uint32_t start, uint32_t lbo, uint32_
   return d;
 }
 
+// The same with 64-byte swizzle (8-row atoms of 512 bytes).
+__device__ inline uint64_t umma_desc_sw64(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;            // SWIZZLE_64B
+  return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                       // D format: f32
@@ -406,6 +443,16 @@ cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStr
 cudaError_t launch_fine_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineTcArgs& a,
                            int num_sms, cudaStream_t s);
 cudaError_t launch_fine_f32(const FineF32Args& a, cudaStream_t s);
+cudaError_t launch_token_pos(const Geom& g, const int* cube_rank, int* pos, cudaStream_t s);
+cudaError_t launch_rope_pairs(const Geom& g, int dt, int dh, int dw, float base, int t_offset, float2* tab,
+                              cudaStream_t s);
+struct QkvTma {
+  int box_rows;    // X rows per tile (the W box is 256 rows)
+  int box_k;       // channels per stage: 64 (128-byte swizzle) or 32 (64-byte swizzle)
+};
+QkvTma qkv_tma(int variant);
+cudaError_t launch_qkv(const CUtensorMap& mx, const CUtensorMap& mw, QkvArgs a, int variant, int num_sms,
+                       cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, long long cap, cudaStream_t s);
 
 }  // namespace fvattn

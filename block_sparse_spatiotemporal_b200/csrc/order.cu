@@ -126,6 +126,18 @@ __global__ void tile_token_kernel(Geom g, const int* cube_rank, int* tile_tok) {
     tile_tok[tiled_position(g, cube_rank, n, bits)] = n;
 }
 
+// pos[n] = tiled row of natural token n.
+__global__ void token_pos_kernel(Geom g, const int* cube_rank, int* pos) {
+  const int bits = hilbert_bits_for(g);
+  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < g.N; n += gridDim.x * blockDim.x)
+    pos[n] = tiled_position(g, cube_rank, n, bits);
+}
+
+cudaError_t launch_token_pos(const Geom& g, const int* cube_rank, int* pos, cudaStream_t s) {
+  token_pos_kernel<<<(g.N + 255) / 256, 256, 0, s>>>(g, cube_rank, pos);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tile_token(const Geom& g, const int* cube_rank, int* tile_tok, cudaStream_t s) {
   tile_token_kernel<<<(g.N + 255) / 256, 256, 0, s>>>(g, cube_rank, tile_tok);
   return cudaGetLastError();

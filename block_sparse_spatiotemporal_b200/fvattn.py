@@ -22,7 +22,7 @@ __all__ = [
     "pool_select_subblock",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
-    "STAGES", "pool_select_noalloc",
+    "STAGES", "pool_select_noalloc", "workspace_size_qkv", "qkv_rope",
 ]
 
 F32, BF16 = 0, 1
@@ -96,6 +96,10 @@ _SIGS = {
                        ctypes.POINTER(Rope), ctypes.c_float, ctypes.c_int32, ctypes.POINTER(MaskCache),
                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                        ctypes.c_void_p],
+    "fvattn_workspace_size_qkv": [ctypes.POINTER(Shape), ctypes.POINTER(Rope), ctypes.POINTER(ctypes.c_size_t)],
+    "fvattn_qkv_rope": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                        ctypes.POINTER(Rope), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_get_device_status": [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)],
     "fvattn_selftest_wait_timeout": [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_void_p],
     "fvattn_profile_enable": [ctypes.c_int],
@@ -103,7 +107,7 @@ _SIGS = {
     "fvattn_status_string": [ctypes.c_int],
 }
 
-STAGES = ("tables", "reorder", "pool", "select", "schedule", "fine")
+STAGES = ("tables", "reorder", "pool", "select", "schedule", "fine", "prologue")
 
 
 def lib():
@@ -288,6 +292,29 @@ def forward(shape: Shape, q, k, v, ws, top_p: float, k_min: int, rope: Optional[
                                 1 if reuse_mask else 0, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                 _stream(stream)))
     return out, lse
+
+
+def workspace_size_qkv(shape: Shape, rope: Optional[Rope] = None) -> int:
+    n = ctypes.c_size_t()
+    _check("fvattn_workspace_size_qkv",
+           lib().fvattn_workspace_size_qkv(ctypes.byref(shape), _rope_ptr(rope), ctypes.byref(n)))
+    return n.value
+
+
+def qkv_rope(shape: Shape, x, w, ws, bias=None, rope: Optional[Rope] = None, t_offset: int = 0, out=None,
+             stream=None):
+    """Prologue: x [B, N, C] bf16, w [3*H*d, C] bf16, bias [3*H*d] float32
+    or None -> (q, k, v) [B, H, N, d] bf16 in shape.layout, Q and K rotated
+    at frame t + t_offset."""
+    B, N, C = x.shape
+    if out is None:
+        out = tuple(torch.empty((shape.batch, shape.heads, N, shape.head_dim), dtype=torch.bfloat16,
+                                device=x.device) for _ in range(3))
+    q, k, v = out
+    _check("fvattn_qkv_rope",
+           lib().fvattn_qkv_rope(ctypes.byref(shape), _ptr(x), int(C), _ptr(w), _ptr(bias), _rope_ptr(rope),
+                                 int(t_offset), _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel(), _stream(stream)))
+    return q, k, v
 
 
 def device_status(ws, stream=None) -> int:

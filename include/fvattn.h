@@ -204,6 +204,33 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
                    int reuse_mask, void* out, float* lse, void* ws, size_t ws_bytes,
                    fvattn_stream_t stream);
 
+/* Attention prologue ("Causal-RoPE SP" digest, section 2.3: the QKV
+ * projection and the rotary encoding fused into one kernel; section 2.2: a
+ * block that starts at frame s encodes its local frame t at global frame
+ * t + s, so a rank needs only s to rotate its own tokens).
+ *   x     [B, N, C] bf16, natural token order (row n = token (t, h, w)).
+ *   w     [3*H*d, C] bf16, a linear layer's weight (output rows first):
+ *         rows 0..H*d-1 project Q (head h at rows h*d..h*d+d-1), then K,
+ *         then V.
+ *   bias  [3*H*d] float32, or NULL for none.
+ *   For every token and output row o: y = sum_c x[n, c] * w[o, c] with fp32
+ *   accumulation of the exact bf16 products, plus bias[o]; with rope
+ *   enabled the Q and K head slices are rotated as in fvattn_rope at
+ *   coordinates (t + t_offset, h, w) in fp32; every result is rounded once
+ *   to bf16.  q, k, v [B, H, N, d] bf16 receive the three parts in
+ *   shape->layout: natural, or tiled in shape->order (the layout
+ *   fvattn_tile_reorder produces), ready for fvattn_pool_select and
+ *   fvattn_block_sparse_fwd.
+ * Requirements: shape->dtype FVATTN_BF16 and head_dim 128; channels a
+ * multiple of 64 in [64, 65536]; 0 <= t_offset <= 2^20; x, w, bias, q, k, v
+ * 16-byte aligned, q, k, v not overlapping x, w or each other.  The
+ * workspace is fvattn_workspace_size_qkv bytes (tables only: N + 2 nT int32
+ * and the (cos, sin) pairs). */
+int fvattn_workspace_size_qkv(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes);
+int fvattn_qkv_rope(const fvattn_shape* shape, const void* x, int32_t channels, const void* w,
+                    const float* bias, const fvattn_rope* rope, int32_t t_offset, void* q, void* k,
+                    void* v, void* ws, size_t ws_bytes, fvattn_stream_t stream);
+
 /* Synchronises the stream, reads and clears the workspace status word.
  * *status is 0 or a positive code: 1 bad block id, 2 wait cap reached. */
 int fvattn_get_device_status(void* ws, fvattn_stream_t stream, int32_t* status);
@@ -229,7 +256,8 @@ typedef enum {
   FVATTN_STAGE_SELECT = 3,    /* coarse scores, softmax, top-p selection */
   FVATTN_STAGE_SCHEDULE = 4,  /* union lists + work-list sort */
   FVATTN_STAGE_FINE = 5,      /* block-sparse fine attention */
-  FVATTN_STAGE_COUNT = 6
+  FVATTN_STAGE_PROLOGUE = 6,  /* fused QKV projection + RoPE */
+  FVATTN_STAGE_COUNT = 7
 } fvattn_stage;
 int fvattn_profile_enable(int enable);
 int fvattn_profile_read(double* ms, int64_t* launches);

@@ -238,7 +238,7 @@ def project_qkv(x, w, bias=None):
 
 
 def qkv_rope(x, w, bias, grid, heads, head_dim, rope=None, t_offset=0,
-             order=None, tokens=None, rounded=True):
+             order=None, tokens=None, rounded=True, gathered=False):
     """The attention prologue ("Causal-RoPE SP" digest, section 2.3: QKV
     projection and the rotary encoding as one operator; section 2.2: a token
     at local frame t of a block that starts at frame s is encoded at global
@@ -251,17 +251,21 @@ def qkv_rope(x, w, bias, grid, heads, head_dim, rope=None, t_offset=0,
     once to bf16.  Returns q, k, v [B, H, N, d] in natural order, or in the
     tiled order ``order`` ("raster" / "hilbert") when given.  ``tokens``
     (natural indices) restricts the result to those tokens, returned as
-    [B, H, len(tokens), d] in the given order (``order`` must then be None)."""
+    [B, H, len(tokens), d] in the given order (``order`` must then be None);
+    with ``gathered`` x holds only those tokens' rows, [B, len(tokens), C]."""
     x = np.asarray(x, np.float64)
-    B, N, _ = x.shape
+    B = x.shape[0]
+    N = grid[0] * grid[1] * grid[2]
     H, d = heads, head_dim
+    if gathered and tokens is None:
+        raise ValueError("gathered needs tokens")
     if tokens is None:
         tok = np.arange(N)
     else:
         if order is not None:
             raise ValueError("tokens and order are exclusive")
         tok = np.asarray(tokens, np.int64)
-    y = project_qkv(x[:, tok, :], w, bias)                   # [B, n, 3*H*d]
+    y = project_qkv(x if gathered else x[:, tok, :], w, bias)  # [B, n, 3*H*d]
     y = y.reshape(B, len(tok), 3, H, d).transpose(2, 0, 3, 1, 4)  # [3, B, H, n, d]
     q, k, v = y[0].copy(), y[1].copy(), y[2].copy()
     if rope is not None:

@@ -122,8 +122,10 @@ def test_tiled_order_token_subset_and_rounding():
             assert np.array_equal(c[..., pos, :], a)
     toks = np.array([0, 5, 77, 255])
     sub = O.qkv_rope(x, w, b, grid, H, d, ROPE, t_offset=1, tokens=toks)
-    for a, c in zip(nat, sub):
+    gat = O.qkv_rope(x[:, toks], w, b, grid, H, d, ROPE, t_offset=1, tokens=toks, gathered=True)
+    for a, c, g in zip(nat, sub, gat):
         assert np.array_equal(c, a[..., toks, :])
+        assert np.array_equal(g, c)
     raw = O.qkv_rope(x, w, b, grid, H, d, ROPE, t_offset=1, rounded=False)
     for a, r in zip(nat, raw):
         assert np.array_equal(a, O.round_bf16(r))
