@@ -35,7 +35,9 @@ Readings where the pages are silent (each also listed in the design notes):
     coarse logit (the probability order, without the ties that underflowing
     probabilities would create), ties to the lower tile index;
     count = min(nT, max(m, k_min)); p >= 1 keeps every tile;
-  * the output is the fine stage only (the coarse stage only routes);
+  * the output is the fine stage only (the coarse stage only routes); so the
+    backward pass is the gradient of the fine stage for fixed lists (the
+    selection is piecewise constant in Q and K and passes no gradient);
   * lse is the natural log of the softmax normaliser;
   * RoPE: per-axis groups of 44/42/42 head dims for (t, h, w), adjacent pairs
     (2j, 2j+1) inside each group, angle = pos * base^(-2j/d_axis); pooling uses
@@ -482,6 +484,85 @@ def fine_head(q_tiled, k_tiled, v_tiled, counts, idx, scale, rows=None, tile_tok
         out[sl], lse[sl] = fine_tile(q_tiled[sl], k_tiled, v_tiled,
                                      idx[i, :counts[i]], scale, tile_tokens)
     return out, lse
+
+
+# ----------------------------------------------------------------------------
+# backward pass of the fine stage
+# ----------------------------------------------------------------------------
+
+def fine_tile_backward(q_tile, k_tiled, v_tiled, do_tile, tiles, scale, tile_tokens=64):
+    """Gradients of L = sum(out * dout) for the 64 query rows of one tile
+    attending over the tokens of the given key tiles ("VSA" digest, section 3:
+    the fine stage is token-level softmax attention inside the selected tiles;
+    it is trained end to end, which needs these gradients).
+
+    With s = scale * q k^T, p = softmax_rows(s), out = p v:
+      dv = p^T dout,  dp = dout v^T,  ds = p * (dp - rowsum(p * dp)),
+      dq = scale * ds k,  dk = scale * ds^T q.
+    Returns (dq [64, d], rows, dk [len(rows), d], dv [len(rows), d]) where
+    ``rows`` are the key token rows the tile attends to (tiled order)."""
+    rows = (np.asarray(tiles)[:, None] * tile_tokens + np.arange(tile_tokens)[None, :]).ravel()
+    q = np.asarray(q_tile, np.float64)
+    ks = np.asarray(k_tiled[rows], np.float64)
+    vs = np.asarray(v_tiled[rows], np.float64)
+    g = np.asarray(do_tile, np.float64)
+    s = scale * (q @ ks.T)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    dv = p.T @ g
+    dp = g @ vs.T
+    ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    return scale * (ds @ ks), rows, scale * (ds.T @ q), dv
+
+
+def fine_head_backward(q_tiled, k_tiled, v_tiled, do_tiled, counts, idx, scale, tile_tokens=64):
+    """dq, dk, dv [N, d] of one head in tiled order: each query tile's
+    gradients (``fine_tile_backward``), the key and value parts summed over
+    every query tile that selected the key's tile.  A query tile with an empty
+    list has zero output and contributes nothing."""
+    N, d = q_tiled.shape
+    dq = np.zeros((N, d))
+    dk = np.zeros((N, d))
+    dv = np.zeros((N, d))
+    for i in range(N // tile_tokens):
+        if counts[i] == 0:
+            continue
+        sl = slice(i * tile_tokens, (i + 1) * tile_tokens)
+        gq, rows, gk, gv = fine_tile_backward(q_tiled[sl], k_tiled, v_tiled, do_tiled[sl],
+                                              idx[i, :counts[i]], scale, tile_tokens)
+        dq[sl] = gq
+        np.add.at(dk, rows, gk)
+        np.add.at(dv, rows, gv)
+    return dq, dk, dv
+
+
+def fine_head_backward_scales(q_tiled, k_tiled, v_tiled, do_tiled, out_tiled, counts, idx, scale,
+                              tile_tokens=64):
+    """Magnitude of the terms behind each gradient element, the scale of the
+    rounding error of any evaluation that rounds p and ds to bf16:
+    with a_rk = p_rk * (|dp_rk| + sum_c |dout_rc * out_rc|),
+      dq: scale * a |k|,  dk: scale * a^T |q|,  dv: p^T |dout|."""
+    N, d = q_tiled.shape
+    sq = np.zeros((N, d))
+    sk = np.zeros((N, d))
+    sv = np.zeros((N, d))
+    for i in range(N // tile_tokens):
+        if counts[i] == 0:
+            continue
+        sl = slice(i * tile_tokens, (i + 1) * tile_tokens)
+        rows = (np.asarray(idx[i, :counts[i]])[:, None] * tile_tokens + np.arange(tile_tokens)[None, :]).ravel()
+        q = np.asarray(q_tiled[sl], np.float64)
+        ks = np.asarray(k_tiled[rows], np.float64)
+        vs = np.asarray(v_tiled[rows], np.float64)
+        g = np.asarray(do_tiled[sl], np.float64)
+        s = scale * (q @ ks.T)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        a = p * (np.abs(g @ vs.T) + np.abs(g * np.asarray(out_tiled[sl], np.float64)).sum(axis=1, keepdims=True))
+        sq[sl] = scale * (a @ np.abs(ks))
+        np.add.at(sk, rows, scale * (a.T @ np.abs(q)))
+        np.add.at(sv, rows, p.T @ np.abs(g))
+    return sq, sk, sv
 
 
 # ----------------------------------------------------------------------------
