@@ -572,6 +572,138 @@ def run_prologue(args, wl):
     return 0
 
 
+def run_backward(args, wl):
+    """The fine-stage backward at the workload's shape: lists from the
+    library's own selection, out / lse from its forward, a seeded dout, all
+    in the tiled layout; one step = one fvattn_block_sparse_bwd call (both
+    schedules, D, the dK/dV and dQ kernels).  Effective FLOP/s counts the five
+    products of the gradient, 5 * 2 * 64 * 64 * d per selected pair."""
+    import torch
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+    from block_sparse_spatiotemporal_b200.inputs import f32_to_bf16_bits
+
+    dev = torch.device("cuda", 0)
+    B, H, N, d = wl.batch, wl.heads, wl.tokens, wl.head_dim
+    q, k, v = make_inputs(wl)
+    g = f32_to_bf16_bits(np.random.default_rng(wl.seed + 77).standard_normal((B, H, N, d), dtype=np.float32))
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    order = F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE
+    nat = F.make_shape(B, H, d, wl.grid, dtype=F.BF16, order=order, layout=F.NATURAL)
+    shape = F.make_shape(B, H, d, wl.grid, dtype=F.BF16, order=order, layout=F.TILED)
+    rope = F.make_rope(wl.rope_dims, wl.rope_base) if wl.rope else None
+    ws = torch.empty(max(F.workspace_size(shape, rope), F.workspace_size_bwd(shape)), dtype=torch.uint8, device=dev)
+    qt, kt, vt = (F.tile_reorder(nat, as_dev(x), ws) for x in (q, k, v))
+    gd = as_dev(g)
+    counts, idx = F.pool_select(shape, qt, kt, ws, wl.top_p, wl.k_min, rope=rope)
+    if rope is not None:   # the backward takes the rotated q, k the fine stage consumed
+        raise SystemExit("--backward takes workloads without RoPE")
+    out, lse = F.block_sparse_fwd(shape, qt, kt, vt, counts, idx, ws)
+    grads = tuple(torch.empty_like(qt) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+    pairs = int(counts.sum().item())
+    flops = 5.0 * 2 * 64 * 64 * d * pairs
+
+    def step():
+        F.block_sparse_bwd(shape, qt, kt, vt, out, gd, lse, counts, idx, ws, grads=grads)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+    sampler = ClockSampler([0])
+    sampler.start()
+    time.sleep(0.3)
+    F.profile_read()
+    F.profile_enable(True)
+    ms = timed(step, args.steps)
+    F.profile_enable(False)
+    stages = F.profile_read()
+    clocks = sampler.stop()
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during the timed region")
+    per = {k: v[0] / max(v[1], 1) for k, v in stages.items() if v[1]}
+    kv_ms, q_ms = per["bwd_kv"], per["bwd_q"]
+    unit_flop = 2.0 * 64 * 64 * d * pairs           # one 64x64xd product per selected pair
+    pk, pk_kind = peaks()
+    kv_ach = 4 * unit_flop / (kv_ms / 1e3) / 1e12   # S^T, dP^T, dV, dK
+    q_ach = 3 * unit_flop / (q_ms / 1e3) / 1e12     # S, dP, dQ
+
+    # end to end: q, k, v, out, dout, lse and the lists from pinned host, dq, dk, dv back
+    hosts = [x.cpu().pin_memory() for x in (qt, kt, vt, out, gd, lse, counts, idx)]
+    devs = [torch.empty_like(x) for x in (qt, kt, vt, out, gd, lse, counts, idx)]
+    ghost = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in grads]
+
+    def e2e_step():
+        for hst, dv_ in zip(hosts, devs):
+            dv_.copy_(hst, non_blocking=True)
+        F.block_sparse_bwd(shape, *devs[:6], devs[6], devs[7], ws, grads=grads)
+        for gr, hst in zip(grads, ghost):
+            hst.copy_(gr, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = timed(e2e_step, max(3, min(args.steps, 10)))
+    big = kv_ms >= q_ms
+    line = {
+        "metric": "fine-stage backward ms & effective TFLOP/s", "value": flops / (ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"backward_{wl.name}", "grid": list(wl.grid), "tokens": N, "heads": H, "head_dim": d,
+                   "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order, "layout": "tiled",
+                   "selected_pairs": pairs, "density": pairs / (H * wl.num_tiles ** 2),
+                   "l2": "inputs larger than L2 (q, k, v, out, dout = %.0f MB)" % (5 * qt.numel() * 2 / 1e6)},
+        "stage_ms": {k: round(v[0] / args.steps, 4) for k, v in stages.items() if v[1]},
+        "kernels": {"bwd_kv": {"ms": kv_ms, "tflops": kv_ach, "products_per_pair": 4},
+                    "bwd_q": {"ms": q_ms, "tflops": q_ach, "products_per_pair": 3}},
+        "roofline": {"kernel": "bwd_tc_kernel<true>" if big else "bwd_tc_kernel<false>", "bound": "tensor",
+                     "achieved": kv_ach if big else q_ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": (kv_ach if big else q_ach) / pk["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{pk_kind} bf16 burst"},
+        "gpu_launches": sum(n for _, n in stages.values()),
+        "clocks": clocks,
+        "e2e": {"value": flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hosts),
+                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in ghost)},
+    }
+    if not args.no_cpu_baseline:
+        from oracle import fvattn_oracle as O
+        rng = np.random.default_rng(0)
+        ch, ih = counts.cpu().numpy()[0], idx.cpu().numpy()[0]
+        pos = O.positions(wl.grid, wl.order)
+        t0 = time.perf_counter()
+        done, rows, cache = 0, 0, {}
+        scale = O.default_scale(d)
+        while time.perf_counter() - t0 < args.cpu_budget or rows == 0:
+            h = int(rng.integers(H))
+            i = int(rng.integers(wl.num_tiles))
+            if h not in cache:   # the head in tiled order (dout is drawn tiled)
+                cache = {h: [O.to_tiled(O.as_f64(x[0, h], "bf16"), pos) for x in (q, k, v)]
+                         + [O.as_f64(g[0, h], "bf16")]}
+            qh, kh, vh, gh = cache[h]
+            sl = slice(64 * i, 64 * i + 64)
+            O.fine_tile_backward(qh[sl], kh, vh, gh[sl], ih[h, i, :ch[h, i]], scale)
+            done += int(ch[h, i])
+            rows += 1
+        el = time.perf_counter() - t0
+        est = el * pairs / max(done, 1)
+        line["cpu_baseline"] = {"value": flops / est / 1e12, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                                "sample": f"oracle (numpy fp64) backward of {rows} random (head, query tile) rows "
+                                          f"({done} selected pairs), scaled by selected pairs",
+                                "est_ms_per_step": est * 1e3}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -586,6 +718,8 @@ def main():
                     help="hierarchical sub-block scoring (pool_select_subblock + block_sparse_fwd)")
     ap.add_argument("--prologue", action="store_true",
                     help="the fused QKV projection + 3D RoPE prologue at the workload's shape (one JSON line)")
+    ap.add_argument("--backward", action="store_true",
+                    help="the fine-stage backward (dq, dk, dv) at the workload's shape (one JSON line)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -595,6 +729,8 @@ def main():
         return run_sweep(args)
     if args.prologue:
         return run_prologue(args, wl)
+    if args.backward:
+        return run_backward(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)

@@ -140,6 +140,32 @@ WsLayout layout_qkv(const Geom& g, const fvattn_rope* r) {
   return L;
 }
 
+// Backward workspace: both schedules, the transposed selection bitmap, D and lse * log2(e).
+WsLayout layout_bwd(const Geom& g) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  const size_t items = (size_t)g.BH * g.P;
+  L.status = take(kAlign);
+  L.uni = take(sizeof(int) * items * g.nT);
+  L.ucount = take(sizeof(int) * items);
+  L.worklist = take(sizeof(int) * items);
+  L.rank = take(sizeof(int) * items);
+  L.bits = take(sizeof(uint32_t) * (size_t)g.BH * g.nT * ((g.nT + 31) / 32));
+  L.uni_t = take(sizeof(int) * items * g.nT);
+  L.ucount_t = take(sizeof(int) * items);
+  L.worklist_t = take(sizeof(int) * items);
+  L.rank_t = take(sizeof(int) * items);
+  L.lse2 = take(sizeof(float) * (size_t)g.BH * g.N);
+  L.dd = take(sizeof(float) * (size_t)g.BH * g.N);
+  L.total = off;
+  return L;
+}
+
 struct DeviceInfo {
   int sms = 0;
   int major = 0;
@@ -325,12 +351,14 @@ int begin(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws,
   return FVATTN_OK;
 }
 
-int begin_qkv(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws, size_t ws_bytes,
-              fvattn_stream_t stream) {
+// As begin(), with the workspace carved by `layout`.
+template <typename F>
+int begin_custom(Call* c, const fvattn_shape* shape, const fvattn_rope* rope, void* ws, size_t ws_bytes,
+                 fvattn_stream_t stream, F layout) {
   FV_TRY(make_geom(shape, &c->g));
   FV_TRY(check_rope(rope, c->g));
   if (!ws || !aligned(ws, kAlign)) return FVATTN_ERR_INVALID_ARG;
-  c->L = layout_qkv(c->g, rope);
+  c->L = layout(c->g);
   if (ws_bytes < c->L.total) return FVATTN_ERR_WORKSPACE;
   FV_TRY(device_info(&c->dev));
   c->ws = static_cast<char*>(ws);
@@ -618,6 +646,79 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
   return FVATTN_OK;
 }
 
+int fvattn_workspace_size_bwd(const fvattn_shape* shape, size_t* bytes) {
+  if (!bytes) return FVATTN_ERR_INVALID_ARG;
+  Geom g{};
+  FV_TRY(make_geom(shape, &g));
+  *bytes = layout_bwd(g).total;
+  return FVATTN_OK;
+}
+
+int fvattn_block_sparse_bwd(const fvattn_shape* shape, const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, const float* lse, const fvattn_blocks* blocks, void* dq, void* dk,
+                            void* dv, void* ws, size_t ws_bytes, fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(out) || !tensor_ok(dout) || !tensor_ok(lse) ||
+      !tensor_ok(dq) || !tensor_ok(dk) || !tensor_ok(dv))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!shape) return FVATTN_ERR_INVALID_ARG;
+  if (shape->dtype != FVATTN_BF16) return FVATTN_ERR_DTYPE;
+  if (shape->layout != FVATTN_LAYOUT_TILED) return FVATTN_ERR_UNSUPPORTED;
+  Call c;
+  FV_TRY(begin_custom(&c, shape, nullptr, ws, ws_bytes, stream, [](const Geom& g) { return layout_bwd(g); }));
+  FV_TRY(check_blocks(blocks, c.g));
+  const Geom& g = c.g;
+  {
+    StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
+    FV_CUDA(launch_union(g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
+                         c.status, c.s));
+    FV_CUDA(launch_rank(c.at<int>(c.L.ucount), g.BH * g.P, c.at<int>(c.L.rank), c.at<int>(c.L.worklist), c.s));
+    FV_CUDA(launch_key_union(g, blocks->counts, blocks->idx, blocks->cap, c.at<uint32_t>(c.L.bits),
+                             c.at<int>(c.L.uni_t), c.at<int>(c.L.ucount_t), c.status, c.s));
+    FV_CUDA(launch_rank(c.at<int>(c.L.ucount_t), g.BH * g.P, c.at<int>(c.L.rank_t), c.at<int>(c.L.worklist_t), c.s));
+    t.kernels = 7;   // union, 2 x (partial ranks, scatter), transpose bits, key union
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  FV_TRY(make_tile_map(&mq, q, g, false));
+  FV_TRY(make_tile_map(&mk, k, g, false));
+  FV_TRY(make_tile_map(&mv, v, g, false));
+  FV_TRY(make_tile_map(&mdo, dout, g, false));
+  {
+    StageTimer t(FVATTN_STAGE_BWD_PREP, c.s);
+    FV_CUDA(launch_bwd_prep(out, dout, lse, c.at<float>(c.L.lse2), c.at<float>(c.L.dd), (long long)g.BH * g.N, c.s));
+    t.kernels = 1;
+  }
+  BwdArgs a{};
+  a.g = g;
+  a.n_items = g.BH * g.P;
+  a.lse2 = c.at<float>(c.L.lse2);
+  a.dd = c.at<float>(c.L.dd);
+  a.scale = g.scale;
+  a.scale_log2 = g.scale * 1.4426950408889634f;
+  a.status = c.status;
+  a.wait_cap = kDefaultWaitCap;
+  // key-stationary: X = (K, V), Y = (Q, dO) -> dK, dV
+  a.uni = c.at<int>(c.L.uni_t);
+  a.ucount = c.at<int>(c.L.ucount_t);
+  a.worklist = c.at<int>(c.L.worklist_t);
+  a.out0 = static_cast<__nv_bfloat16*>(dk);
+  a.out1 = static_cast<__nv_bfloat16*>(dv);
+  {
+    StageTimer t(FVATTN_STAGE_BWD_KV, c.s);
+    FV_CUDA(launch_bwd(mk, mv, mq, mdo, a, true, c.dev.sms, c.s));
+    t.kernels = 1;
+  }
+  // query-stationary: X = (Q, dO), Y = (K, V) -> dQ
+  a.uni = c.at<int>(c.L.uni);
+  a.ucount = c.at<int>(c.L.ucount);
+  a.worklist = c.at<int>(c.L.worklist);
+  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  a.out1 = nullptr;
+  StageTimer t(FVATTN_STAGE_BWD_Q, c.s);
+  FV_CUDA(launch_bwd(mq, mdo, mk, mv, a, false, c.dev.sms, c.s));
+  t.kernels = 1;
+  return FVATTN_OK;
+}
+
 int fvattn_workspace_size_qkv(const fvattn_shape* shape, const fvattn_rope* rope, size_t* bytes) {
   if (!bytes) return FVATTN_ERR_INVALID_ARG;
   Geom g{};
@@ -645,7 +746,7 @@ int fvattn_qkv_rope(const fvattn_shape* shape, const void* x, int32_t channels, 
   if (shape->dtype != FVATTN_BF16) return FVATTN_ERR_DTYPE;
   if (channels < 64 || channels > 65536 || channels % 64) return FVATTN_ERR_SHAPE;
   Call c;
-  FV_TRY(begin_qkv(&c, shape, rope, ws, ws_bytes, stream));
+  FV_TRY(begin_custom(&c, shape, rope, ws, ws_bytes, stream, [&](const Geom& g) { return layout_qkv(g, rope); }));
   const Geom& g = c.g;
   const bool tiled = shape->layout == FVATTN_LAYOUT_TILED;
   const bool r = rope_on(rope);

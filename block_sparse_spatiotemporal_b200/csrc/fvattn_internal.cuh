@@ -59,6 +59,10 @@ struct WsLayout {
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
   size_t skh, skl;       //   ... of K
   size_t tmass;          //   float [BH*nT*8*nT] log2 key-tile masses per query sub-block
+  size_t bits;           // backward only: u32 [BH*nT*ceil(nT/32)] transposed selection bitmap
+  size_t uni_t, ucount_t;  //   union lists of key-tile pairs
+  size_t worklist_t, rank_t;
+  size_t lse2, dd;       //   float [BH*N] lse * log2(e) and rowsum(dout * out)
   size_t tok_pos;        // prologue only: int32 [N] tiled row of natural token n
   size_t rope_pairs;     //   float2 pair-major (cos, sin) table at the start-frame offset
   size_t total;
@@ -110,6 +114,22 @@ struct QkvArgs {
   int Nout;                // 3 * H * 128 rows of W
   int kblocks;             // C / 64
   int mt, nt, n_tiles, group_m;
+  int* status;
+  long long wait_cap;
+};
+
+// Backward of the fine stage (both kernels of the template).
+struct BwdArgs {
+  Geom g;
+  const int* uni;          // union lists of the items (key-stationary: of key-tile pairs)
+  const int* ucount;
+  const int* worklist;
+  int n_items;
+  const float* lse2;       // [BH, N] lse * log2(e), tiled rows
+  const float* dd;         // [BH, N] rowsum(dout * out)
+  __nv_bfloat16* out0;     // dK (key-stationary) or dQ
+  __nv_bfloat16* out1;     // dV (key-stationary)
+  float scale, scale_log2;
   int* status;
   long long wait_cap;
 };
@@ -453,6 +473,12 @@ struct QkvTma {
 QkvTma qkv_tma(int variant);
 cudaError_t launch_qkv(const CUtensorMap& mx, const CUtensorMap& mw, QkvArgs a, int variant, int num_sms,
                        cudaStream_t s);
+cudaError_t launch_bwd_prep(const void* out, const void* dout, const float* lse, float* lse2, float* dd, long long rows,
+                            cudaStream_t s);
+cudaError_t launch_key_union(const Geom& g, const int* counts, const int* idx, int cap, uint32_t* bits, int* uni,
+                             int* ucount, int* status, cudaStream_t s);
+cudaError_t launch_bwd(const CUtensorMap& s0, const CUtensorMap& s1, const CUtensorMap& m0, const CUtensorMap& m1,
+                       const BwdArgs& a, bool key_stationary, int num_sms, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, long long cap, cudaStream_t s);
 
 }  // namespace fvattn

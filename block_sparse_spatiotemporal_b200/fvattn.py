@@ -22,7 +22,7 @@ __all__ = [
     "pool_select_subblock",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
-    "STAGES", "pool_select_noalloc", "workspace_size_qkv", "qkv_rope",
+    "STAGES", "pool_select_noalloc", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
 ]
 
 F32, BF16 = 0, 1
@@ -96,6 +96,11 @@ _SIGS = {
                        ctypes.POINTER(Rope), ctypes.c_float, ctypes.c_int32, ctypes.POINTER(MaskCache),
                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                        ctypes.c_void_p],
+    "fvattn_workspace_size_bwd": [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
+    "fvattn_block_sparse_bwd": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Blocks),
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                ctypes.c_void_p],
     "fvattn_workspace_size_qkv": [ctypes.POINTER(Shape), ctypes.POINTER(Rope), ctypes.POINTER(ctypes.c_size_t)],
     "fvattn_qkv_rope": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                         ctypes.POINTER(Rope), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -107,7 +112,7 @@ _SIGS = {
     "fvattn_status_string": [ctypes.c_int],
 }
 
-STAGES = ("tables", "reorder", "pool", "select", "schedule", "fine", "prologue")
+STAGES = ("tables", "reorder", "pool", "select", "schedule", "fine", "prologue", "bwd_prep", "bwd_kv", "bwd_q")
 
 
 def lib():
@@ -292,6 +297,25 @@ def forward(shape: Shape, q, k, v, ws, top_p: float, k_min: int, rope: Optional[
                                 1 if reuse_mask else 0, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                 _stream(stream)))
     return out, lse
+
+
+def workspace_size_bwd(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check("fvattn_workspace_size_bwd", lib().fvattn_workspace_size_bwd(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def block_sparse_bwd(shape: Shape, q, k, v, out, dout, lse, counts, idx, ws, grads=None, stream=None):
+    """Backward of step 6 (tiled layout, bf16): returns (dq, dk, dv)."""
+    if grads is None:
+        grads = tuple(torch.empty_like(q) for _ in range(3))
+    dq, dk, dv = grads
+    b = _blocks_of(counts, idx)
+    _check("fvattn_block_sparse_bwd",
+           lib().fvattn_block_sparse_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                         _ptr(lse), ctypes.byref(b), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                         ws.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def workspace_size_qkv(shape: Shape, rope: Optional[Rope] = None) -> int:

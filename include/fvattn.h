@@ -204,6 +204,31 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
                    int reuse_mask, void* out, float* lse, void* ws, size_t ws_bytes,
                    fvattn_stream_t stream);
 
+/* Backward pass of step 6 ("VSA" digest, section 3: the fine block-sparse
+ * attention is trained end to end).  For the lists in `blocks` (fixed: the
+ * selection is piecewise constant in q and k and passes no gradient) and
+ * the forward's out and lse, computes the gradients of
+ * L = sum(out * dout): with s = scale q k^T and p = exp(s - lse) over each
+ * row's selected keys,
+ *   dv = p^T dout,  ds = p * (dout v^T - rowsum(dout * out)),
+ *   dq = scale ds k,  dk = scale ds^T q,
+ * summed over every query tile that selected a key's tile (keys no tile
+ * selected get zero gradients; a query tile with an empty list gets dq = 0).
+ * q, k, v, out, dout, dq, dk, dv are [B, H, N, 128] bf16 in the TILED layout
+ * (shape->layout must be FVATTN_LAYOUT_TILED, else FVATTN_ERR_UNSUPPORTED);
+ * lse [B, H, N] float32 as fvattn_block_sparse_fwd wrote it; q and k are the
+ * tensors the fine stage consumed (rotated ones when RoPE was used).  bf16
+ * only (FVATTN_ERR_DTYPE otherwise).  P and dS are rounded to bf16 for the
+ * tensor cores, accumulation is fp32, the gradients are rounded once to bf16.
+ * No atomics: the result is deterministic.  Workspace:
+ * fvattn_workspace_size_bwd bytes.  Bad block ids set status 1 and are
+ * dropped. */
+int fvattn_workspace_size_bwd(const fvattn_shape* shape, size_t* bytes);
+int fvattn_block_sparse_bwd(const fvattn_shape* shape, const void* q, const void* k, const void* v,
+                            const void* out, const void* dout, const float* lse,
+                            const fvattn_blocks* blocks, void* dq, void* dk, void* dv, void* ws,
+                            size_t ws_bytes, fvattn_stream_t stream);
+
 /* Attention prologue ("Causal-RoPE SP" digest, section 2.3: the QKV
  * projection and the rotary encoding fused into one kernel; section 2.2: a
  * block that starts at frame s encodes its local frame t at global frame
@@ -257,7 +282,10 @@ typedef enum {
   FVATTN_STAGE_SCHEDULE = 4,  /* union lists + work-list sort */
   FVATTN_STAGE_FINE = 5,      /* block-sparse fine attention */
   FVATTN_STAGE_PROLOGUE = 6,  /* fused QKV projection + RoPE */
-  FVATTN_STAGE_COUNT = 7
+  FVATTN_STAGE_BWD_PREP = 7,  /* backward: D = rowsum(dout * out), lse * log2(e) */
+  FVATTN_STAGE_BWD_KV = 8,    /* backward: key-stationary dK, dV kernel */
+  FVATTN_STAGE_BWD_Q = 9,     /* backward: query-stationary dQ kernel */
+  FVATTN_STAGE_COUNT = 10
 } fvattn_stage;
 int fvattn_profile_enable(int enable);
 int fvattn_profile_read(double* ms, int64_t* launches);
