@@ -10,51 +10,57 @@
 // atomics:
 //   * key-stationary (KV = true): a work item is two adjacent key tiles of one
 //     head (128 TMEM lanes); it walks the union of the query tiles that
-//     selected either key tile, two query tiles (128 queries) per step, and
+//     selected either key tile, one query tile (64 queries) per step, and
 //     accumulates dV += P^T dO and dK += dS^T Q in TMEM;
 //   * query-stationary (KV = false): a work item is two adjacent query tiles
-//     (the forward's items and union lists); per step two selected key tiles,
+//     (the forward's items and union lists); one selected key tile per step,
 //     accumulating dQ += dS K.
-// Per step one thread issues S = X0 Y0^T and dP = X1 Y1^T (X stationary:
-// K, V or Q, dO; Y moving: Q, dO or K, V) into TMEM; four warps (one TMEM lane
-// per thread) turn them into P and dS, write both back into the same TMEM
-// columns as bf16, and the accumulating MMAs read them from TMEM as the A
-// operand.  The moving tiles are used twice: K-major for the scores,
-// MN-major for the accumulations.  Layout: tiled only.
+// Per step two threads issue S = X0 Y0^T and dP = X1 Y1^T (X stationary:
+// K, V or Q, dO; Y moving: Q, dO or K, V; M128 N64) into one of two TMEM
+// buffers; eight warps (two per TMEM lane quarter, half the columns each)
+// turn them into P and dS and write both back into the same TMEM columns as
+// bf16, and a third thread's accumulating MMAs read them from TMEM as the A
+// operand.  With two S / dP buffers the next step's scores run on the tensor
+// cores while the warps work on this step's.  The moving tiles are used
+// twice: K-major for the scores, MN-major for the accumulations.  Layout:
+// tiled only.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
 namespace bw {
 
-constexpr int THREADS = 256;          // warp 0 TMA, warp 1 MMA, warps 4..7 compute + epilogue
+constexpr int THREADS = 384;          // warp 0 TMA, warps 1-3 MMA, warps 4..11 compute + epilogue
 constexpr int CW0 = 4;
+constexpr int CTHREADS = 256;         // compute threads: two warps per TMEM lane quarter
 constexpr uint32_t BOX = 64 * 128;    // 64 rows x 128 bytes
-constexpr uint32_t HALF = 2 * BOX;    // one 64-dim half of 128 rows: 16 KB
+constexpr uint32_t HALF = 2 * BOX;    // one 64-dim half of the 128 stationary rows: 16 KB
 constexpr uint32_t TENSOR = 4 * BOX;  // 128 rows x 128 dims bf16: 32 KB
-constexpr int MST = 2;                // moving stages
+constexpr uint32_t MTENSOR = 2 * BOX; // one moving tile, 64 rows x 128 dims: 16 KB (halves BOX apart)
+constexpr int MST = 4;                // moving stages
 constexpr uint32_t STAT_BYTES = 2 * TENSOR;
-constexpr uint32_t MOV_BYTES = 2 * TENSOR;
+constexpr uint32_t MOV_BYTES = 2 * MTENSOR;
 constexpr uint32_t SMEM_BYTES = 1024 + STAT_BYTES + MST * MOV_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
+// S buffer b at columns 64 b, dP buffer b at 128 + 64 b; accumulators at 256 and 384
 constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 384;
-constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
-constexpr int STEP_LAST = 1 << 4;     // step word: sel of moving tile 0 (bits 0-1), tile 1 (2-3), last
+constexpr int STEP_LAST = 1 << 4;     // step word: sel of the moving tile (bits 0-1), last
 static_assert(SMEM_BYTES + 3 * 1024 <= 227 * 1024, "shared memory");
 
 struct Ctl {
   uint64_t stat_full, stat_empty;
   uint64_t mov_full[MST], mov_empty[MST];
-  uint64_t s_full;      // S and dP of the step in TMEM (commit) + step word written (MMA thread)
-  uint64_t p_full;      // P / dS written back (128 compute threads)
-  uint64_t step_done;   // the step's accumulating MMAs complete (they read P / dS)
+  uint64_t s_full[2];   // S and dP of step c in buffer c & 1 (two commits) + step word written
+  uint64_t p_full[2];   // P / dS of step c written back (256 compute threads)
+  uint64_t step_done[2];// the accumulating MMAs of step c, which read buffer c & 1, complete
   uint64_t acc_full;    // the item's accumulators complete
-  uint64_t acc_empty;   // the epilogue read them (128 threads)
+  uint64_t acc_empty;   // the epilogue read them (256 threads)
   uint64_t drain;
   int meta[MST];        // step word per moving stage
-  int info;             // step word of the step in TMEM
-  float lse2[MST][128]; // key-stationary only: lse * log2(e) of the step's queries
-  float dd[MST][128];   //   and their D
+  int info[2];          // step word of the step in each buffer
+  float lse2[MST][64];  // key-stationary only: lse * log2(e) of the step's queries
+  float dd[MST][64];    //   and their D
   uint32_t tmem_base;
   int abort;
 };
@@ -79,16 +85,17 @@ __device__ inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
       : "memory");
 }
 
-// Both 64-dim halves of one 64-row tile of a tiled [BH, N, 128] tensor into
-// rows 0..63 (slot 0) or 64..127 (slot 1) of a 128-row operand.
-__device__ inline void load_tile(const CUtensorMap* map, int bh, int tile, uint8_t* base, int slot, uint64_t* bar) {
-  tma_load_3d(base + slot * BOX, map, bar, 0, tile * kTileTokens, bh);
-  tma_load_3d(base + slot * BOX + HALF, map, bar, 64, tile * kTileTokens, bh);
+// Both 64-dim halves of one 64-row tile of a tiled [BH, N, 128] tensor, the
+// second half `stride` bytes after the first.
+__device__ inline void load_tile(const CUtensorMap* map, int bh, int tile, uint8_t* dst, uint32_t stride,
+                                 uint64_t* bar) {
+  tma_load_3d(dst, map, bar, 0, tile * kTileTokens, bh);
+  tma_load_3d(dst + stride, map, bar, 64, tile * kTileTokens, bh);
 }
 
-// 128 rows x 128 bytes of a tensor in SMEM (two 16 KB halves), K-major.
-__device__ inline uint64_t kdesc(uint32_t base, int kk) {
-  return umma_desc_sw128(base + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024);
+// K-major operand whose two 64-dim halves are `stride` bytes apart.
+__device__ inline uint64_t kdesc(uint32_t base, uint32_t stride, int kk) {
+  return umma_desc_sw128(base + (kk >> 2) * stride + (kk & 3) * 32, 16, 1024);
 }
 
 template <bool KV>
@@ -109,17 +116,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->stat_full, 1);
-    mbar_init(&ctl->stat_empty, 1);
+    mbar_init(&ctl->stat_empty, 2);      // one commit per score thread
     for (int i = 0; i < MST; ++i) {
       mbar_init(&ctl->mov_full[i], KV ? 32 : 1);
       mbar_init(&ctl->mov_empty[i], 1);
     }
-    mbar_init(&ctl->s_full, 2);
-    mbar_init(&ctl->p_full, 128);
-    mbar_init(&ctl->step_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl->s_full[i], 3);     // two commits + the step word
+      mbar_init(&ctl->p_full[i], CTHREADS);
+      mbar_init(&ctl->step_done[i], 1);
+    }
     mbar_init(&ctl->acc_full, 1);
-    mbar_init(&ctl->acc_empty, 128);
-    mbar_init(&ctl->drain, 1);
+    mbar_init(&ctl->acc_empty, CTHREADS);
+    mbar_init(&ctl->drain, 3);           // final commit of each MMA thread
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -153,10 +162,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (k >= 1) ok = mbar_wait(&ctl->stat_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap);
         if (ok) {
           mbar_arrive_expect_tx(&ctl->stat_full, STAT_BYTES);
-          load_tile(&ms0, bh, t0, sStat, 0, &ctl->stat_full);
-          load_tile(&ms0, bh, t1, sStat, 1, &ctl->stat_full);
-          load_tile(&ms1, bh, t0, sStat + TENSOR, 0, &ctl->stat_full);
-          load_tile(&ms1, bh, t1, sStat + TENSOR, 1, &ctl->stat_full);
+          load_tile(&ms0, bh, t0, sStat, HALF, &ctl->stat_full);
+          load_tile(&ms0, bh, t1, sStat + BOX, HALF, &ctl->stat_full);
+          load_tile(&ms1, bh, t0, sStat + TENSOR, HALF, &ctl->stat_full);
+          load_tile(&ms1, bh, t1, sStat + TENSOR + BOX, HALF, &ctl->stat_full);
           ++stat_issued;
         }
       }
@@ -164,7 +173,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       const int n = a.ucount[item];
       const int* list = a.uni + (size_t)item * g.nT;
-      const int steps = (n + 1) >> 1;
       for (int e0 = 0; e0 < n && ok; e0 += 32) {
         int ent = e0 + lane < n ? list[e0 + lane] : 0;
         if ((ent & 0xFFFF) >= g.nT) {  // never produced by the schedule; keep the copy in bounds
@@ -172,36 +180,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           ent &= ~0x3FFFF;
         }
         const int cnt = n - e0 < 32 ? n - e0 : 32;
-        for (int i = 0; i < cnt; i += 2, ++gs) {
-          const bool two = i + 1 < cnt;
-          const int ent0 = __shfl_sync(0xffffffffu, ent, i);
-          const int ent1 = __shfl_sync(0xffffffffu, ent, two ? i + 1 : i);
-          const int j0 = ent0 & 0xFFFF, j1 = ent1 & 0xFFFF;
+        for (int i = 0; i < cnt; ++i, ++gs) {
+          const int e = __shfl_sync(0xffffffffu, ent, i);
+          const int j = e & 0xFFFF;
           const int st = (int)(gs % MST);
-          const int step = (e0 + i) >> 1;
           if (leader && gs >= MST)
             ok = mbar_wait(&ctl->mov_empty[st], (uint32_t)((gs / MST) - 1) & 1, abort_flag, a.status, cap);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           if (KV) {
-            // the step's 128 queries: lse * log2(e) and D, 4 per lane
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int q = lane * 4 + u;
-              const size_t row = (size_t)bh * g.N + (size_t)(q < 64 ? j0 : j1) * kTileTokens + (q & 63);
-              ctl->lse2[st][q] = a.lse2[row];
-              ctl->dd[st][q] = a.dd[row];
-            }
+            // the step's 64 queries: lse * log2(e) and D, 2 per lane
+            const size_t row = (size_t)bh * g.N + (size_t)j * kTileTokens + 2 * lane;
+            const float2 l2 = *reinterpret_cast<const float2*>(a.lse2 + row);
+            const float2 d2 = *reinterpret_cast<const float2*>(a.dd + row);
+            ctl->lse2[st][2 * lane] = l2.x;
+            ctl->lse2[st][2 * lane + 1] = l2.y;
+            ctl->dd[st][2 * lane] = d2.x;
+            ctl->dd[st][2 * lane + 1] = d2.y;
           }
           if (leader) {
-            ctl->meta[st] = ((ent0 >> 16) & 3) | (two ? ((ent1 >> 16) & 3) << 2 : 0) |
-                            (step == steps - 1 ? STEP_LAST : 0);
+            ctl->meta[st] = ((e >> 16) & 3) | ((e0 + i == n - 1) ? STEP_LAST : 0);
             mbar_arrive_expect_tx(&ctl->mov_full[st], MOV_BYTES);
             uint8_t* dst = sMov + st * MOV_BYTES;
-            load_tile(&mm0, bh, j0, dst, 0, &ctl->mov_full[st]);
-            load_tile(&mm0, bh, j1, dst, 1, &ctl->mov_full[st]);
-            load_tile(&mm1, bh, j0, dst + TENSOR, 0, &ctl->mov_full[st]);
-            load_tile(&mm1, bh, j1, dst + TENSOR, 1, &ctl->mov_full[st]);
+            load_tile(&mm0, bh, j, dst, BOX, &ctl->mov_full[st]);
+            load_tile(&mm1, bh, j, dst + MTENSOR, BOX, &ctl->mov_full[st]);
           } else if (KV) {
             mbar_arrive(&ctl->mov_full[st]);
           }
@@ -216,72 +218,97 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_drain(&ctl->mov_full[i], (uint32_t)(last / MST) & 1, a.status, cap);
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // ------------------------------------------------------- MMA: scores
+    // Warp 1 issues S = X0 Y0^T, warp 2 dP = X1 Y1^T (one thread issues a
+    // tcgen05.mma only every ~100 clk, about what an N=64 MMA takes to run,
+    // so the step's MMAs are spread over three threads).  Step c goes to
+    // buffer c & 1 once the accumulations of step c - 2, which read it, are
+    // complete; the stationary tiles are released after the item's last score.
+    const bool is_s = warp == 1;
     long long c = 0;
     int k = 0;
     bool ok = true;
-    const uint32_t s0 = smem_u32(sStat), s1 = s0 + TENSOR;
+    const uint32_t x = smem_u32(sStat) + (is_s ? 0u : TENSOR);
+    const uint32_t tdst = tbase + (is_s ? T_S : T_DP);
     for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
       if (!mbar_wait(&ctl->stat_full, (uint32_t)k & 1, abort_flag, a.status, cap)) break;
-      if (k >= 1 && !mbar_wait(&ctl->acc_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) break;
-      tc_fence_after();
-      bool first = true;
       while (true) {
         const int st = (int)(c % MST);
-        if (!mbar_wait(&ctl->mov_full[st], (uint32_t)(c / MST) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        // S and dP overwrite the P / dS the previous step's accumulations read
-        if (c >= 1 && !mbar_wait(&ctl->step_done, (uint32_t)(c - 1) & 1, abort_flag, a.status, cap)) {
+        const int b = (int)(c & 1);
+        if (!mbar_wait(&ctl->mov_full[st], (uint32_t)(c / MST) & 1, abort_flag, a.status, cap) ||
+            (c >= 2 && !mbar_wait(&ctl->step_done[b], (uint32_t)((c - 2) >> 1) & 1, abort_flag, a.status, cap))) {
           ok = false;
           break;
         }
         const int meta = ctl->meta[st];
-        ctl->info = meta;
+        if (is_s) ctl->info[b] = meta;
         tc_fence_after();
-        const uint32_t y0 = smem_u32(sMov + st * MOV_BYTES), y1 = y0 + TENSOR;
+        const uint32_t y = smem_u32(sMov + st * MOV_BYTES) + (is_s ? 0u : MTENSOR);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tbase + T_S, kdesc(s0, kk), kdesc(y0, kk), IDESC_S, kk ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tbase + T_DP, kdesc(s1, kk), kdesc(y1, kk), IDESC_S, kk ? 1u : 0u);
-        mma_commit(&ctl->s_full);
-        mbar_arrive(&ctl->s_full);
-        if (!mbar_wait(&ctl->p_full, (uint32_t)c & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // 16 moving rows = 16 operand rows of 128 bytes per K step; P / dS of moving row 16 kk in
-        // TMEM columns 8 kk .. 8 kk + 7 (bf16 pairs)
-        const uint64_t b0 = umma_desc_sw128(y0, HALF, 1024), b1 = umma_desc_sw128(y1, HALF, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          if (KV) {
-            mma_ts(tbase + T_ACC1, tbase + T_S + 8 * kk, b1 + ((kk * 2048) >> 4), IDESC_ACC, acc);   // dV
-            mma_ts(tbase + T_ACC0, tbase + T_DP + 8 * kk, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dK
-          } else {
-            mma_ts(tbase + T_ACC0, tbase + T_DP + 8 * kk, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dQ
-          }
-        }
-        mma_commit(&ctl->mov_empty[st]);
-        mma_commit(&ctl->step_done);
-        first = false;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tdst + 64 * b, kdesc(x, HALF, kk), kdesc(y, BOX, kk), IDESC_S, kk ? 1u : 0u);
+        mma_commit(&ctl->s_full[b]);
+        if (is_s) mbar_arrive(&ctl->s_full[b]);
         ++c;
         if (meta & STEP_LAST) break;
       }
       if (!ok) break;
-      mma_commit(&ctl->acc_full);
       mma_commit(&ctl->stat_empty);
     }
     // every MMA issued has completed before TMEM is freed
     mma_commit(&ctl->drain);
     mbar_drain(&ctl->drain, 0, a.status, cap);
+  } else if (warp == 3 && lane == 0) {
+    // ------------------------------------------------- MMA: accumulations
+    long long c = 0;
+    int k = 0;
+    bool ok = true;
+    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+      if (k >= 1 && !mbar_wait(&ctl->acc_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) break;
+      bool first = true;
+      while (true) {
+        const int b = (int)(c & 1);
+        const int st = (int)(c % MST);
+        if (!mbar_wait(&ctl->p_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        const int info = ctl->info[b];
+        tc_fence_after();
+        // 16 moving rows = 2048 bytes of the MN-major operand per K step; P / dS of moving rows
+        // 16 kk .. 16 kk + 15 in TMEM columns 32 (kk / 2) + 8 (kk % 2) .. + 7 of the buffer
+        // (bf16 pairs; each 32-row half packed at the start of its own 32 columns)
+        const uint32_t y0 = smem_u32(sMov + st * MOV_BYTES), y1 = y0 + MTENSOR;
+        const uint64_t b0 = umma_desc_sw128(y0, BOX, 1024), b1 = umma_desc_sw128(y1, BOX, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          const uint32_t col = 64 * b + 32 * (kk >> 1) + 8 * (kk & 1);
+          if (KV) {
+            mma_ts(tbase + T_ACC1, tbase + T_S + col, b1 + ((kk * 2048) >> 4), IDESC_ACC, acc);   // dV
+            mma_ts(tbase + T_ACC0, tbase + T_DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dK
+          } else {
+            mma_ts(tbase + T_ACC0, tbase + T_DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dQ
+          }
+        }
+        mma_commit(&ctl->mov_empty[st]);
+        mma_commit(&ctl->step_done[b]);
+        first = false;
+        ++c;
+        if (info & STEP_LAST) break;
+      }
+      if (!ok) break;
+      mma_commit(&ctl->acc_full);
+    }
+    mma_commit(&ctl->drain);
+    mbar_drain(&ctl->drain, 0, a.status, cap);
   } else if (warp >= CW0) {
     // ------------------------------------------------- P, dS and epilogue
+    // warps 4..7 take moving columns 0..31 of every step and accumulator
+    // columns 0..63, warps 8..11 the other half
     const int q4 = warp & 3;
+    const int part = (warp - CW0) >> 2;
     const int r = q4 * 32 + lane;                 // TMEM lane = row of the item
     const int h = r >> 6;                         // stationary tile of the row
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
@@ -301,22 +328,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       bool ok = true;
       while (true) {
-        if (!mbar_wait(&ctl->s_full, (uint32_t)c & 1, abort_flag, a.status, cap)) {
+        const int b = (int)(c & 1);
+        if (!mbar_wait(&ctl->s_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
-        const int info = ctl->info;
+        const int info = ctl->info[b];
         const int st = (int)(c % MST);
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          const int t = ch >> 1;
-          const bool on = (((info >> (2 * t)) & 3) >> h) & 1;     // uniform across the warp
+        const bool on = ((info & 3) >> h) & 1;       // uniform across the warp
+        const uint32_t tS = tbase + T_S + 64 * b + lane_off, tD = tbase + T_DP + 64 * b + lane_off;
+        {
+          const int ch = part;
           uint32_t pk[16], dk[16];
           if (on) {
             uint32_t s[32], dp[32];
-            tmem_ld32(tbase + T_S + lane_off + 32 * ch, s);
-            tmem_ld32(tbase + T_DP + lane_off + 32 * ch, dp);
+            tmem_ld32(tS + 32 * ch, s);
+            tmem_ld32(tD + 32 * ch, dp);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -336,12 +364,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = dk[i] = 0u;
           }
-          if (KV) tmem_st16(tbase + T_S + lane_off + 16 * ch, pk);
-          tmem_st16(tbase + T_DP + lane_off + 16 * ch, dk);
+          // packed into the first 16 of the 32 columns this warp read (the other
+          // warp of the lane quarter reads and writes only its own 32)
+          if (KV) tmem_st16(tS + 32 * ch, pk);
+          tmem_st16(tD + 32 * ch, dk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->p_full);
+        mbar_arrive(&ctl->p_full[b]);
         ++c;
         if (info & STEP_LAST) break;
       }
@@ -355,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float mul = o == 0 ? a.scale : 1.f;      // dq, dk carry the softmax scale; dv does not
         __nv_bfloat16* dst = (o == 0 ? a.out0 : a.out1) + row * 128;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 2 * part; ch < 2 * part + 2; ++ch) {
           uint32_t v[32];
           tmem_ld32(tacc + 32 * ch, v);
           tmem_wait_ld();
