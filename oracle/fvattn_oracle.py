@@ -54,6 +54,10 @@ Readings where the pages are silent (each also listed in the design notes):
     key sub-blocks of j (the sum of the fine scores, normalised so that each
     row sums to one); top-p and k_min then act on these tile probabilities,
     ranked by their logarithm (no underflow ties);
+  * timestep schedule: optional dense first steps, then (top_p, k_min)
+    linear in the step from their start to their end values;
+  * slack-aware augmentation: see ``augment_lists`` (the persistent fine
+    stage's CTAs play the pages' ranks; costs are union entries);
   * prologue: Q | K | V = X W^T + b, one linear layer whose 3*H*d output
     rows are Q heads, then K heads, then V heads (head h of each at rows
     h*d..h*d+d-1); Q and K are rotated by the 3D RoPE above at
@@ -484,6 +488,103 @@ def fine_head(q_tiled, k_tiled, v_tiled, counts, idx, scale, rows=None, tile_tok
         out[sl], lse[sl] = fine_tile(q_tiled[sl], k_tiled, v_tiled,
                                      idx[i, :counts[i]], scale, tile_tokens)
     return out, lse
+
+
+# ----------------------------------------------------------------------------
+# timestep schedule and slack-aware augmentation
+# ----------------------------------------------------------------------------
+
+def timestep_params(step, num_steps, p_start, p_end, k_start, k_end, dense_steps=0):
+    """(top_p, k_min) for diffusion step ``step`` of ``num_steps`` ("DFSAttn"
+    digest, section 3: sparsity is low while the frames are still noise and
+    rises as the video sharpens).  The first ``dense_steps`` steps keep every
+    tile (top_p = 1); over the remaining steps top_p and k_min move linearly
+    from (p_start, k_start) to (p_end, k_end), k_min rounded half up."""
+    if step < dense_steps:
+        return 1.0, int(k_start)
+    span = num_steps - dense_steps - 1
+    f = 0.0 if span <= 0 else (step - dense_steps) / span
+    f = min(max(f, 0.0), 1.0)
+    p = p_start + (p_end - p_start) * f
+    k = int(math.floor(k_start + (k_end - k_start) * f + 0.5))
+    return p, k
+
+
+def item_unions(counts, idx, nT):
+    """Key-tile union of each work item (query tiles 2q, 2q+1 of one head):
+    counts [BH, nT], idx [BH, nT, cap] -> list over items (b*H + h)*P + q of
+    sets; the item's cost is max(1, len(set)) (an empty union still takes one
+    masked step)."""
+    BH = counts.shape[0]
+    P = (nT + 1) // 2
+    out = []
+    for bh in range(BH):
+        for q in range(P):
+            u = set()
+            for r in (2 * q, 2 * q + 1):
+                if r < nT:
+                    u.update(int(j) for j in idx[bh, r, :counts[bh, r]])
+            out.append(u)
+    return out
+
+
+def lpt_order(costs):
+    """Items by cost descending, ties by ascending item code."""
+    return sorted(range(len(costs)), key=lambda i: (-costs[i], i))
+
+
+def augment_lists(S, counts, idx, num_ctas):
+    """Slack-aware augmentation on one GPU ("FVAttn" digest, section 02: ranks
+    off the critical path spend their spare time on extra, somewhat
+    important blocks), with the persistent fine stage's CTAs as the ranks.
+
+    The work list is the longest-first order of the items' union costs; CTA c
+    of ``num_ctas`` runs the items at slots c, c + G, ...; its slack is the
+    largest CTA load minus its own.  The slack is split evenly over the CTA's
+    items (the first ones in slot order take the remainder); an item receives
+    that many extra key tiles, at most the tiles outside its union, only if
+    one of its rows has a list: the outside tiles with the largest logit max
+    over the item's rows with a list (ties to the lower tile), added to each
+    of those rows.  S [BH, nT, nT] are the coarse logits.
+
+    Returns (counts, idx, extra, worklist): the augmented lists (ascending),
+    the tiles added per item, and the work list the fine stage keeps (the
+    order of the unaugmented costs)."""
+    BH, nT = counts.shape
+    P = (nT + 1) // 2
+    unions = item_unions(counts, idx, nT)
+    costs = [max(1, len(u)) for u in unions]
+    order = lpt_order(costs)
+    G = max(1, min(num_ctas, len(order)))
+    loads = [sum(costs[order[t]] for t in range(c, len(order), G)) for c in range(G)]
+    top = max(loads)
+    extra = [0] * len(order)
+    for c in range(G):
+        slots = list(range(c, len(order), G))
+        slack, n = top - loads[c], len(slots)
+        for u, t in enumerate(slots):
+            extra[order[t]] = slack // n + (1 if u < slack % n else 0)
+    new_counts = counts.copy()
+    new_idx = np.zeros((BH, nT, nT), dtype=idx.dtype)
+    for bh in range(BH):
+        for r in range(nT):
+            new_idx[bh, r, :counts[bh, r]] = idx[bh, r, :counts[bh, r]]
+    added = [0] * len(order)
+    for item in range(len(order)):
+        bh, q = divmod(item, P)
+        rows = [r for r in (2 * q, 2 * q + 1) if r < nT and counts[bh, r] > 0]
+        e = min(extra[item], nT - len(unions[item])) if rows else 0
+        if e <= 0:
+            continue
+        cand = [j for j in range(nT) if j not in unions[item]]
+        score = {j: max(S[bh, r, j] for r in rows) for j in cand}
+        pick = sorted(cand, key=lambda j: (-score[j], j))[:e]
+        added[item] = len(pick)
+        for r in rows:
+            lst = sorted(set(int(j) for j in idx[bh, r, :counts[bh, r]]) | set(pick))
+            new_counts[bh, r] = len(lst)
+            new_idx[bh, r, :len(lst)] = lst
+    return new_counts, new_idx, added, order
 
 
 # ----------------------------------------------------------------------------
