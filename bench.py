@@ -704,6 +704,77 @@ def run_backward(args, wl):
     return 0
 
 
+def run_augment(args, wl):
+    """Slack-aware augmentation at the workload's shape: the plain path
+    (selection, schedule, fine stage) against selection, augmentation to one
+    CTA per SM and the fine stage on the kept work list; one JSON line with
+    both times, the selected pairs before and after, and the fine-stage times."""
+    import torch
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+
+    dev = torch.device("cuda", 0)
+    q, k, v = make_inputs(wl)
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
+    shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16,
+                         order=F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE)
+    rope = F.make_rope(wl.rope_dims, wl.rope_base) if wl.rope else None
+    ws = F.workspace(shape, rope, device=dev)
+    G = torch.cuda.get_device_properties(dev).multi_processor_count
+    base = F.new_blocks(shape, dev)
+    aug = F.new_blocks(shape, dev)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def plain():
+        F.pool_select(shape, qd, kd, ws, wl.top_p, wl.k_min, rope=rope, blocks=base)
+        F.block_sparse_fwd(shape, qd, kd, vd, base[0], base[1], ws, rope=rope, out=out, lse=lse)
+
+    def augmented():
+        F.pool_select(shape, qd, kd, ws, wl.top_p, wl.k_min, rope=rope, blocks=base)
+        _, _, wlist = F.augment_lists(shape, qd, kd, ws, base[0], base[1], num_ctas=G, rope=rope,
+                                      out=(aug[0], aug[1]))
+        F.block_sparse_fwd_worklist(shape, qd, kd, vd, aug[0], aug[1], wlist, ws, num_ctas=G, rope=rope,
+                                    out=out, lse=lse)
+
+    res = {}
+    for name, fn in (("plain", plain), ("augmented", augmented)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        F.profile_read()
+        F.profile_enable(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        F.profile_enable(False)
+        st = F.profile_read()
+        if F.device_status(ws) != 0:
+            raise RuntimeError("device status set")
+        res[name] = {"ms": e0.elapsed_time(e1) / args.steps,
+                     "fine_ms": st["fine"][0] / max(st["fine"][1], 1),
+                     "stage_ms": {k2: round(v2[0] / args.steps, 4) for k2, v2 in st.items() if v2[1]}}
+    pairs = int(base[0].sum().item())
+    apairs = int(aug[0].sum().item())
+    fl = pair_flops(wl.head_dim)
+    line = {"metric": "slack-aware augmentation: sparse-attn fwd ms & effective TFLOP/s", "unit": UNIT,
+            "value": apairs * fl / (res["augmented"]["ms"] / 1e3) / 1e12, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["augmented"]["ms"], "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"augment_{wl.name}", "grid": list(wl.grid), "heads": wl.heads,
+                       "top_p": wl.top_p, "k_min": wl.k_min, "ctas": G},
+            "selected_pairs": {"plain": pairs, "augmented": apairs, "added": apairs - pairs},
+            "plain": res["plain"], "augmented": res["augmented"],
+            "fine_tflops": {"plain": pairs * fl / (res["plain"]["fine_ms"] / 1e3) / 1e12,
+                            "augmented": apairs * fl / (res["augmented"]["fine_ms"] / 1e3) / 1e12}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -720,6 +791,8 @@ def main():
                     help="the fused QKV projection + 3D RoPE prologue at the workload's shape (one JSON line)")
     ap.add_argument("--backward", action="store_true",
                     help="the fine-stage backward (dq, dk, dv) at the workload's shape (one JSON line)")
+    ap.add_argument("--augment", action="store_true",
+                    help="slack-aware augmentation against the plain path at the workload's shape (one JSON line)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -731,6 +804,8 @@ def main():
         return run_prologue(args, wl)
     if args.backward:
         return run_backward(args, wl)
+    if args.augment:
+        return run_augment(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_gpu(args, wl)

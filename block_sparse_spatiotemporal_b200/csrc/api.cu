@@ -412,6 +412,8 @@ int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const vo
   FV_TRY(make_pooled_map(&mkl, po.lo[1], c.g));
   ScoreArgs sa{c.g, c.at<float>(c.L.scores), c.status, kDefaultWaitCap};
   FV_CUDA(launch_scores(mqh, mql, mkh, mkl, sa, c.s));
+  t.kernels = 1;
+  if (!blocks) return FVATTN_OK;   // coarse logits only
   FV_CUDA(launch_select(c.g, sa.S, top_p, k_min, blocks->counts, blocks->idx, blocks->cap, c.s));
   t.kernels = 2;
   return FVATTN_OK;
@@ -427,8 +429,11 @@ int run_schedule(const Call& c, const fvattn_blocks* blocks, int* worklist) {
 }
 
 // Fine stage.  q/k come from the rotated tiled copies when RoPE is on.
+// worklist / grid: a caller's work list and persistent grid (default: the
+// schedule's work list in the workspace and one CTA per SM).
 int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const void* v,
-             const fvattn_rope* rope, bool natural, const fvattn_blocks* blocks, void* out, float* lse) {
+             const fvattn_rope* rope, bool natural, const fvattn_blocks* blocks, void* out, float* lse,
+             const int* worklist = nullptr, int grid = 0) {
   const bool r = rope_on(rope);
   const void* qs = r ? c.at<void>(c.L.qrot) : q;
   const void* ks = r ? c.at<void>(c.L.krot) : k;
@@ -442,7 +447,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.g = c.g;
     a.uni = c.at<int>(c.L.uni);
     a.ucount = c.at<int>(c.L.ucount);
-    a.worklist = c.at<int>(c.L.worklist);
+    a.worklist = worklist ? worklist : c.at<int>(c.L.worklist);
     a.n_items = c.g.BH * c.g.P;
     a.tile_cube = c.at<int>(c.L.tile_cube);
     a.q_nat = qk_nat;
@@ -454,7 +459,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.status = c.status;
     a.wait_cap = kDefaultWaitCap;
     StageTimer t(FVATTN_STAGE_FINE, c.s);
-    FV_CUDA(launch_fine_tc(mq, mk, mv, a, c.dev.sms, c.s));
+    FV_CUDA(launch_fine_tc(mq, mk, mv, a, grid > 0 ? grid : c.dev.sms, c.s));
     t.kernels = a.n_items > 0 ? 1 : 0;
   } else {
     FineF32Args a{};
@@ -605,6 +610,71 @@ int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void
   if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
   FV_TRY(run_schedule(c, blocks, c.at<int>(c.L.worklist)));
   FV_TRY(run_fine(c, shape, q, k, v, rope, natural, blocks, out, lse));
+  return FVATTN_OK;
+}
+
+int fvattn_augment_lists(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
+                         const fvattn_blocks* base, int32_t num_ctas, const fvattn_blocks* out, int32_t* worklist,
+                         void* ws, size_t ws_bytes, fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !worklist || !aligned(worklist, 4)) return FVATTN_ERR_INVALID_ARG;
+  if (num_ctas < 0 || num_ctas > 1024) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream));
+  FV_TRY(check_blocks(base, c.g));
+  FV_TRY(check_blocks(out, c.g));
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
+  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, false, 0.f, 0, nullptr));
+  FV_TRY(run_schedule(c, base, worklist));
+  const int items = c.g.BH * c.g.P;
+  int G = num_ctas > 0 ? num_ctas : c.dev.sms;
+  if (G > items) G = items;
+  if (G > 1024) G = 1024;
+  StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
+  // the rank buffer is free once the work list is built: it holds the per-item extra tiles
+  FV_CUDA(launch_augment(c.g, c.at<float>(c.L.scores), base->counts, base->idx, base->cap, c.at<int>(c.L.ucount),
+                         worklist, G, c.at<int>(c.L.rank), out->counts, out->idx, out->cap, c.status, c.s));
+  t.kernels = 2;
+  return FVATTN_OK;
+}
+
+int fvattn_block_sparse_fwd_worklist(const fvattn_shape* shape, const void* q, const void* k, const void* v,
+                                     const fvattn_rope* rope, const fvattn_blocks* blocks, const int32_t* worklist,
+                                     int32_t num_ctas, void* out, float* lse, void* ws, size_t ws_bytes,
+                                     fvattn_stream_t stream) {
+  if (!tensor_ok(q) || !tensor_ok(k) || !tensor_ok(v) || !tensor_ok(out) || !lse || !aligned(lse, 4))
+    return FVATTN_ERR_INVALID_ARG;
+  if (!worklist || !aligned(worklist, 4) || num_ctas < 0) return FVATTN_ERR_INVALID_ARG;
+  Call c;
+  FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream));
+  FV_TRY(check_blocks(blocks, c.g));
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
+  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
+  {
+    StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
+    FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
+                         c.status, c.s));
+    t.kernels = 1;
+  }
+  FV_TRY(run_fine(c, shape, q, k, v, rope, natural, blocks, out, lse, worklist, num_ctas));
+  return FVATTN_OK;
+}
+
+int fvattn_timestep_params(int32_t step, int32_t num_steps, float p_start, float p_end, int32_t k_start,
+                           int32_t k_end, int32_t dense_steps, float* top_p, int32_t* k_min) {
+  if (!top_p || !k_min || num_steps < 1 || step < 0 || step >= num_steps || dense_steps < 0) return FVATTN_ERR_INVALID_ARG;
+  if (std::isnan(p_start) || std::isnan(p_end) || k_start < 0 || k_end < 0) return FVATTN_ERR_INVALID_ARG;
+  if (step < dense_steps) {
+    *top_p = 1.f;
+    *k_min = k_start;
+    return FVATTN_OK;
+  }
+  const int span = num_steps - dense_steps - 1;
+  double f = span <= 0 ? 0.0 : (double)(step - dense_steps) / span;
+  f = f < 0.0 ? 0.0 : (f > 1.0 ? 1.0 : f);
+  *top_p = (float)(p_start + (p_end - (double)p_start) * f);
+  *k_min = (int32_t)std::floor(k_start + (k_end - (double)k_start) * f + 0.5);
   return FVATTN_OK;
 }
 

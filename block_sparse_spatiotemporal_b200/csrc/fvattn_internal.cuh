@@ -479,6 +479,9 @@ cudaError_t launch_key_union(const Geom& g, const int* counts, const int* idx, i
                              int* ucount, int* status, cudaStream_t s);
 cudaError_t launch_bwd(const CUtensorMap& s0, const CUtensorMap& s1, const CUtensorMap& m0, const CUtensorMap& m1,
                        const BwdArgs& a, bool key_stationary, int num_sms, cudaStream_t s);
+cudaError_t launch_augment(const Geom& g, const float* S, const int* counts, const int* idx, int cap,
+                           const int* ucount, const int* worklist, int G, int* extra, int* out_counts, int* out_idx,
+                           int out_cap, int* status, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, long long cap, cudaStream_t s);
 
 }  // namespace fvattn

@@ -23,6 +23,7 @@ __all__ = [
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
     "STAGES", "pool_select_noalloc", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
+    "augment_lists", "block_sparse_fwd_worklist", "timestep_params",
 ]
 
 F32, BF16 = 0, 1
@@ -96,6 +97,16 @@ _SIGS = {
                        ctypes.POINTER(Rope), ctypes.c_float, ctypes.c_int32, ctypes.POINTER(MaskCache),
                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                        ctypes.c_void_p],
+    "fvattn_augment_lists": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
+                             ctypes.POINTER(Blocks), ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p,
+                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+    "fvattn_block_sparse_fwd_worklist": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.POINTER(Rope), ctypes.POINTER(Blocks), ctypes.c_void_p,
+                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.c_void_p],
+    "fvattn_timestep_params": [ctypes.c_int32, ctypes.c_int32, ctypes.c_float, ctypes.c_float, ctypes.c_int32,
+                               ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_float),
+                               ctypes.POINTER(ctypes.c_int32)],
     "fvattn_workspace_size_bwd": [ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
     "fvattn_block_sparse_bwd": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Blocks),
@@ -297,6 +308,49 @@ def forward(shape: Shape, q, k, v, ws, top_p: float, k_min: int, rope: Optional[
                                 1 if reuse_mask else 0, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                 _stream(stream)))
     return out, lse
+
+
+def augment_lists(shape: Shape, q, k, ws, counts, idx, num_ctas: int = 0, rope: Optional[Rope] = None, out=None,
+                  stream=None):
+    """Slack-aware augmentation of (counts, idx): returns (counts, idx,
+    worklist) -- the augmented lists and the work list to run them with."""
+    if out is None:
+        oc, oi, ob = new_blocks(shape, q.device)
+    else:
+        oc, oi = out
+        ob = _blocks_of(oc, oi)
+    wl = torch.empty(shape.batch * shape.heads * ((num_tiles(shape) + 1) // 2), dtype=torch.int32, device=q.device)
+    base = _blocks_of(counts, idx)
+    _check("fvattn_augment_lists",
+           lib().fvattn_augment_lists(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope), ctypes.byref(base),
+                                      int(num_ctas), ctypes.byref(ob), _ptr(wl), _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+    return oc, oi, wl
+
+
+def block_sparse_fwd_worklist(shape: Shape, q, k, v, counts, idx, worklist, ws, num_ctas: int = 0,
+                              rope: Optional[Rope] = None, out=None, lse=None, stream=None):
+    """Step 6 with a given work list and persistent grid: returns (out, lse)."""
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    b = _blocks_of(counts, idx)
+    _check("fvattn_block_sparse_fwd_worklist",
+           lib().fvattn_block_sparse_fwd_worklist(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _rope_ptr(rope),
+                                                  ctypes.byref(b), _ptr(worklist), int(num_ctas), _ptr(out),
+                                                  _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def timestep_params(step: int, num_steps: int, p_start: float, p_end: float, k_start: int, k_end: int,
+                    dense_steps: int = 0):
+    """(top_p, k_min) of a diffusion step (host arithmetic in the library)."""
+    p = ctypes.c_float()
+    km = ctypes.c_int32()
+    _check("fvattn_timestep_params",
+           lib().fvattn_timestep_params(int(step), int(num_steps), float(p_start), float(p_end), int(k_start),
+                                        int(k_end), int(dense_steps), ctypes.byref(p), ctypes.byref(km)))
+    return p.value, km.value
 
 
 def workspace_size_bwd(shape: Shape) -> int:

@@ -204,6 +204,48 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
                    int reuse_mask, void* out, float* lse, void* ws, size_t ws_bytes,
                    fvattn_stream_t stream);
 
+/* Slack-aware augmentation on one GPU ("FVAttn" digest, section 02: ranks
+ * off the critical path spend their spare time on extra, somewhat important
+ * blocks).  The persistent fine stage's CTAs play the ranks.  From the lists
+ * in `base` (selected by any means; shape->layout as in fvattn_pool_select),
+ * builds the fine stage's work list (fvattn_build_worklist's order) into
+ * `worklist` [B*H*P] and assumes CTA c of G = min(num_ctas, B*H*P) runs the
+ * slots c, c + G, ...; an item costs its union size (at least 1).  Each CTA's
+ * slack (the largest CTA load minus its own) is split evenly over its items,
+ * the first in slot order taking the remainder; an item with at least one
+ * non-empty row then adds up to that many key tiles outside its union, by
+ * the largest coarse logit over its non-empty rows (ties to the lower tile
+ * id; logits as fvattn_pool_select computes them, with rope), to each of
+ * those rows.  Writes the augmented lists (ascending) to `out`, which may be
+ * `base` itself.  Run the fine stage with fvattn_block_sparse_fwd_worklist
+ * and the same worklist and num_ctas so that the critical path keeps its
+ * length.  num_ctas in [0, 1024], 0 = the device's SM count (the fine
+ * stage's grid). */
+int fvattn_augment_lists(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
+                         const fvattn_blocks* base, int32_t num_ctas, const fvattn_blocks* out,
+                         int32_t* worklist, void* ws, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Step 6 with a caller's work list (B*H*P item codes, each once) and
+ * persistent grid of num_ctas CTAs (0 = the SM count); otherwise as
+ * fvattn_block_sparse_fwd.  fp32 workloads ignore the work list. */
+int fvattn_block_sparse_fwd_worklist(const fvattn_shape* shape, const void* q, const void* k,
+                                     const void* v, const fvattn_rope* rope,
+                                     const fvattn_blocks* blocks, const int32_t* worklist,
+                                     int32_t num_ctas, void* out, float* lse, void* ws,
+                                     size_t ws_bytes, fvattn_stream_t stream);
+
+/* Timestep schedule of the selection ("DFSAttn" digest, section 3: sparsity
+ * is low while the frames are still noise and rises as the video sharpens).
+ * Host-only arithmetic, no device call.  For diffusion step `step` of
+ * `num_steps`: the first `dense_steps` steps keep every tile (*top_p = 1,
+ * *k_min = k_start); over the remaining steps top_p and k_min move linearly
+ * from (p_start, k_start) to (p_end, k_end), k_min rounded half up.  Feed
+ * the result to fvattn_forward (a cache refilled when the lists should
+ * follow the new sparsity). */
+int fvattn_timestep_params(int32_t step, int32_t num_steps, float p_start, float p_end,
+                           int32_t k_start, int32_t k_end, int32_t dense_steps, float* top_p,
+                           int32_t* k_min);
+
 /* Backward pass of step 6 ("VSA" digest, section 3: the fine block-sparse
  * attention is trained end to end).  For the lists in `blocks` (fixed: the
  * selection is piecewise constant in q and k and passes no gradient) and
