@@ -371,7 +371,10 @@ def run_gpu(args, wl):
                                 "in its loads"},
             "roofline": {"kernel": "fine_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{pk_kind} bf16 burst"},
+                         "peak_source": f"{pk_kind} bf16 burst",
+                         "peak_sustained": pk.get("bf16_tflops_sustained"),
+                         "frac_sustained": achieved / pk["bf16_tflops_sustained"]
+                         if pk.get("bf16_tflops_sustained") else None},
             "gpu_launches": sum(n for _, n in stages.values()),
             "clocks": clocks,
             "e2e": e2e,
