@@ -802,7 +802,7 @@ int fvattn_workspace_size_qkv(const fvattn_shape* shape, const fvattn_rope* rope
 #define FVATTN_QKV_VARIANT 1   // 128 x 256 tiles, double-buffered accumulators
 #endif
 #ifndef FVATTN_QKV_GROUP_M
-#define FVATTN_QKV_GROUP_M 8
+#define FVATTN_QKV_GROUP_M 16   // row tiles per band (16 beat 4, 8 and 32 at 720p)
 #endif
 
 int fvattn_qkv_rope(const fvattn_shape* shape, const void* x, int32_t channels, const void* w, const float* bias,
