@@ -138,3 +138,35 @@ def test_status_strings(lib):
     for code in range(-9, 1):
         assert lib.fvattn_status_string(code)
     assert b"unknown" in lib.fvattn_status_string(42)
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
+    """Prologue, backward and augmentation: argument, dtype, layout and shape
+    errors are returned before any device call (fake aligned pointers)."""
+    al = ctypes.c_void_p(0x100000)
+    s = F.make_shape(1, 1, 128, (4, 4, 8), layout=F.TILED)
+    # prologue: null input, channels not a multiple of 64, negative start frame, fp32
+    assert lib.fvattn_qkv_rope(ctypes.byref(s), None, 64, al, None, None, 0, al, al, al, al, 1 << 20, None) == -1
+    assert lib.fvattn_qkv_rope(ctypes.byref(s), al, 96, al, None, None, 0, al, al, al, al, 1 << 20, None) == -2
+    assert lib.fvattn_qkv_rope(ctypes.byref(s), al, 64, al, None, None, -1, al, al, al, al, 1 << 20, None) == -1
+    f32 = F.make_shape(1, 1, 128, (4, 4, 8), dtype=F.F32, layout=F.TILED)
+    assert lib.fvattn_qkv_rope(ctypes.byref(f32), al, 64, al, None, None, 0, al, al, al, al, 1 << 20, None) == -3
+    # backward: natural layout is not built, fp32 is not a backward dtype, null gradient
+    b = F.Blocks(al.value, al.value, 2)
+    nat = F.make_shape(1, 1, 128, (4, 4, 8))
+    args = (al, al, al, al, al, ctypes.cast(al, ctypes.c_void_p), ctypes.byref(b), al, al, al, al, 1 << 30, None)
+    assert lib.fvattn_block_sparse_bwd(ctypes.byref(nat), *args) == -9
+    assert lib.fvattn_block_sparse_bwd(ctypes.byref(f32), *args) == -3
+    assert lib.fvattn_block_sparse_bwd(ctypes.byref(s), al, al, al, al, al, al, ctypes.byref(b), None, al, al, al,
+                                       1 << 30, None) == -1
+    # augmentation: more than 1024 CTAs, null work list
+    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 2048, ctypes.byref(b), al, al,
+                                    1 << 30, None) == -1
+    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 0, ctypes.byref(b), None, al,
+                                    1 << 30, None) == -1
+    assert lib.fvattn_block_sparse_fwd_worklist(ctypes.byref(s), al, al, al, None, ctypes.byref(b), None, 0, al, al,
+                                                al, 1 << 30, None) == -1
+    # workspace sizes of the new entry points
+    n = ctypes.c_size_t()
+    assert lib.fvattn_workspace_size_bwd(ctypes.byref(s), ctypes.byref(n)) == 0 and n.value > 0
+    assert lib.fvattn_workspace_size_qkv(ctypes.byref(s), None, ctypes.byref(n)) == 0 and n.value > 0
