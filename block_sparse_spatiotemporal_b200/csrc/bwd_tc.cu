@@ -16,14 +16,15 @@
 //     (the forward's items and union lists); one selected key tile per step,
 //     accumulating dQ += dS K.
 // Per step two threads issue S = X0 Y0^T and dP = X1 Y1^T (X stationary:
-// K, V or Q, dO; Y moving: Q, dO or K, V; M128 N64) into one of two TMEM
-// buffers; eight warps (two per TMEM lane quarter, half the columns each)
-// turn them into P and dS and write both back into the same TMEM columns as
-// bf16, and a third thread's accumulating MMAs read them from TMEM as the A
-// operand.  With two S / dP buffers the next step's scores run on the tensor
-// cores while the warps work on this step's.  The moving tiles are used
-// twice: K-major for the scores, MN-major for the accumulations.  Layout:
-// tiled only.
+// K, V or Q, dO; Y moving: Q, dO or K, V; M128 N64) into one of NB TMEM
+// buffers (two in the key-stationary kernel, three in the query-stationary
+// one, which has a single accumulator); eight warps (two per TMEM lane
+// quarter, half the columns each) turn them into P and dS and write both
+// back into the same TMEM columns as bf16, and a third thread's accumulating
+// MMAs read them from TMEM as the A operand.  With several buffers the next
+// steps' scores run on the tensor cores while the warps work on this step's.
+// The moving tiles are used twice: K-major for the scores, MN-major for the
+// accumulations.  Layout: tiled only.
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
@@ -41,8 +42,15 @@ constexpr uint32_t STAT_BYTES = 2 * TENSOR;
 constexpr uint32_t MOV_BYTES = 2 * MTENSOR;
 constexpr uint32_t SMEM_BYTES = 1024 + STAT_BYTES + MST * MOV_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
-// S buffer b at columns 64 b, dP buffer b at 128 + 64 b; accumulators at 256 and 384
-constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 384;
+// NB score buffers: S buffer b at columns 64 b, dP buffer b at 64 (NB + b), then the
+// accumulators (128 columns each).  The key-stationary kernel has two accumulators and
+// room for two buffers, the query-stationary kernel one accumulator and three buffers.
+template <bool KV> struct Tm {
+  static constexpr int NB = KV ? 2 : 3;
+  static constexpr uint32_t S = 0, DP = 64 * NB, ACC0 = 128 * NB, ACC1 = ACC0 + 128;
+  static_assert(ACC0 + (KV ? 256 : 128) <= TMEM_COLS, "TMEM columns");
+};
+constexpr int MAXNB = 3;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
 constexpr int STEP_LAST = 1 << 4;     // step word: sel of the moving tile (bits 0-1), last
@@ -51,14 +59,14 @@ static_assert(SMEM_BYTES + 3 * 1024 <= 227 * 1024, "shared memory");
 struct Ctl {
   uint64_t stat_full, stat_empty;
   uint64_t mov_full[MST], mov_empty[MST];
-  uint64_t s_full[2];   // S and dP of step c in buffer c & 1 (two commits) + step word written
-  uint64_t p_full[2];   // P / dS of step c written back (256 compute threads)
-  uint64_t step_done[2];// the accumulating MMAs of step c, which read buffer c & 1, complete
+  uint64_t s_full[MAXNB];   // S and dP of step c in buffer c % NB (two commits) + step word written
+  uint64_t p_full[MAXNB];   // P / dS of step c written back (256 compute threads)
+  uint64_t step_done[MAXNB];// the accumulating MMAs of step c, which read buffer c % NB, complete
   uint64_t acc_full;    // the item's accumulators complete
   uint64_t acc_empty;   // the epilogue read them (256 threads)
   uint64_t drain;
   int meta[MST];        // step word per moving stage
-  int info[2];          // step word of the step in each buffer
+  int info[MAXNB];      // step word of the step in each buffer
   float lse2[MST][64];  // key-stationary only: lse * log2(e) of the step's queries
   float dd[MST][64];    //   and their D
   uint32_t tmem_base;
@@ -121,7 +129,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&ctl->mov_full[i], KV ? 32 : 1);
       mbar_init(&ctl->mov_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < MAXNB; ++i) {
       mbar_init(&ctl->s_full[i], 3);     // two commits + the step word
       mbar_init(&ctl->p_full[i], CTHREADS);
       mbar_init(&ctl->step_done[i], 1);
@@ -223,21 +231,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Warp 1 issues S = X0 Y0^T, warp 2 dP = X1 Y1^T (one thread issues a
     // tcgen05.mma only every ~100 clk, about what an N=64 MMA takes to run,
     // so the step's MMAs are spread over three threads).  Step c goes to
-    // buffer c & 1 once the accumulations of step c - 2, which read it, are
+    // buffer c % NB once the accumulations of step c - NB, which read it, are
     // complete; the stationary tiles are released after the item's last score.
     const bool is_s = warp == 1;
     long long c = 0;
     int k = 0;
     bool ok = true;
     const uint32_t x = smem_u32(sStat) + (is_s ? 0u : TENSOR);
-    const uint32_t tdst = tbase + (is_s ? T_S : T_DP);
+    const uint32_t tdst = tbase + (is_s ? Tm<KV>::S : Tm<KV>::DP);
     for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
       if (!mbar_wait(&ctl->stat_full, (uint32_t)k & 1, abort_flag, a.status, cap)) break;
       while (true) {
         const int st = (int)(c % MST);
-        const int b = (int)(c & 1);
+        constexpr int NB = Tm<KV>::NB;
+        const int b = (int)(c % NB);
         if (!mbar_wait(&ctl->mov_full[st], (uint32_t)(c / MST) & 1, abort_flag, a.status, cap) ||
-            (c >= 2 && !mbar_wait(&ctl->step_done[b], (uint32_t)((c - 2) >> 1) & 1, abort_flag, a.status, cap))) {
+            (c >= NB && !mbar_wait(&ctl->step_done[b], (uint32_t)((c - NB) / NB) & 1, abort_flag, a.status, cap))) {
           ok = false;
           break;
         }
@@ -268,9 +277,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (k >= 1 && !mbar_wait(&ctl->acc_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) break;
       bool first = true;
       while (true) {
-        const int b = (int)(c & 1);
+        constexpr int NB = Tm<KV>::NB;
+        const int b = (int)(c % NB);
         const int st = (int)(c % MST);
-        if (!mbar_wait(&ctl->p_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+        if (!mbar_wait(&ctl->p_full[b], (uint32_t)(c / NB) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
@@ -286,10 +296,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t acc = (first && kk == 0) ? 0u : 1u;
           const uint32_t col = 64 * b + 32 * (kk >> 1) + 8 * (kk & 1);
           if (KV) {
-            mma_ts(tbase + T_ACC1, tbase + T_S + col, b1 + ((kk * 2048) >> 4), IDESC_ACC, acc);   // dV
-            mma_ts(tbase + T_ACC0, tbase + T_DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dK
+            mma_ts(tbase + Tm<KV>::ACC1, tbase + Tm<KV>::S + col, b1 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dV
+            mma_ts(tbase + Tm<KV>::ACC0, tbase + Tm<KV>::DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc); // dK
           } else {
-            mma_ts(tbase + T_ACC0, tbase + T_DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc);  // dQ
+            mma_ts(tbase + Tm<KV>::ACC0, tbase + Tm<KV>::DP + col, b0 + ((kk * 2048) >> 4), IDESC_ACC, acc); // dQ
           }
         }
         mma_commit(&ctl->mov_empty[st]);
@@ -328,8 +338,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       bool ok = true;
       while (true) {
-        const int b = (int)(c & 1);
-        if (!mbar_wait(&ctl->s_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+        constexpr int NB = Tm<KV>::NB;
+        const int b = (int)(c % NB);
+        if (!mbar_wait(&ctl->s_full[b], (uint32_t)(c / NB) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = (int)(c % MST);
         tc_fence_after();
         const bool on = ((info & 3) >> h) & 1;       // uniform across the warp
-        const uint32_t tS = tbase + T_S + 64 * b + lane_off, tD = tbase + T_DP + 64 * b + lane_off;
+        const uint32_t tS = tbase + Tm<KV>::S + 64 * b + lane_off, tD = tbase + Tm<KV>::DP + 64 * b + lane_off;
         {
           const int ch = part;
           uint32_t pk[16], dk[16];
@@ -381,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
 #pragma unroll 1
       for (int o = 0; o < (KV ? 2 : 1); ++o) {
-        const uint32_t tacc = tbase + (o == 0 ? T_ACC0 : T_ACC1) + lane_off;
+        const uint32_t tacc = tbase + (o == 0 ? Tm<KV>::ACC0 : Tm<KV>::ACC1) + lane_off;
         const float mul = o == 0 ? a.scale : 1.f;      // dq, dk carry the softmax scale; dv does not
         __nv_bfloat16* dst = (o == 0 ? a.out0 : a.out1) + row * 128;
 #pragma unroll 1
