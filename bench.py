@@ -212,6 +212,24 @@ def run_reference(args, wl):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's time: every rank takes part (a collective), so the
+    job's time is the max.  A single rank returns its own time."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Weak scaling: every rank processes the same units; value = all ranks'
+    units / the slowest rank's time (per second), in 1e12 units."""
+    return world * units_per_rank / (ms_max / 1e3) / 1e12
+
+
 def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
@@ -277,10 +295,7 @@ def run_gpu(args, wl):
     ms = e0.elapsed_time(e1) / args.steps
     if F.device_status(ws) != 0:
         raise RuntimeError("device status set during the timed region")
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev, world)
 
     # ---- end to end through the public API: pinned host in, host out
     e2e = None
@@ -304,13 +319,10 @@ def run_gpu(args, wl):
             oh.copy_(out, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        t2 = torch.tensor([s0.elapsed_time(s1) / n_e2e], device=dev)
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t2.item())
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev, world)
         h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
         d2h = oh.numel() * oh.element_size()
-        e2e = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e = {"value": whole_job_value(world, flops_step, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- the tile reorder as its own pass (the forward folds it into its loads): q, k, v to
@@ -344,7 +356,7 @@ def run_gpu(args, wl):
         qk_bytes = 2 * wl.heads * wl.tokens * wl.head_dim * 2
         line = {
             "metric": METRIC,
-            "value": world * flops_step / (ms_max / 1e3) / 1e12,
+            "value": whole_job_value(world, flops_step, ms_max),
             "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps,
