@@ -17,14 +17,21 @@ Sources (page title, section):
     predicts per-tile importance, the fine stage runs token-level attention
     only inside the selected tiles.
   * "FVAttn" digest (iselia-ai.com), sections 00 and 02: the routing front end
-    is top-p routing with a top-k safety floor.
+    is top-p routing with a top-k safety floor; ranks off the critical path
+    spend spare time on extra, somewhat important blocks (slack-aware
+    augmentation).
+  * "VSA" digest, section 3, also: the coarse and fine stages are trained end
+    to end (hence the fine stage's backward pass).
   * "DFSAttn" digest (gist.science 2605.23445), section 1 "Hilbert shuffle":
     tokens are reordered along a 3D Hilbert curve before blocking; section 2
     "sub-block scores": a block is split into smaller sub-blocks, each scored,
     and the fine scores are summed into the block's importance; section 3
-    "smart cache": the previous step's selection is reused.
+    "smart cache": the previous step's selection is reused, and sparsity is
+    low at the early, noisy steps and rises as the video sharpens.
   * "Causal-RoPE SP" digest (gist.science 2603.06664), sections 2.2-2.3: 3D
-    rotary position encoding with precomputed frequencies.
+    rotary position encoding with precomputed frequencies, the global frame
+    index t + s of a block starting at frame s, and the QKV projection fused
+    with the rotation.
 
 Readings where the pages are silent (each also listed in the design notes):
   * pooling is the mean over the 64 tokens of a tile;

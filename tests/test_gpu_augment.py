@@ -70,6 +70,7 @@ def compare(wl, counts, idx, S, tol, G, gc, gi, gw):
     dict(grid=(8, 16, 24), heads=4, G=3, p=0.9, k_min=2),
     dict(grid=(8, 16, 24), heads=4, G=16, p=0.8, k_min=1, order="hilbert", rope=True),
     dict(grid=(4, 8, 12), heads=2, G=200, p=0.5, k_min=1),        # more CTAs than items
+    dict(grid=(4, 4, 20), heads=3, G=2, p=0.6, k_min=1),          # nT = 5: the last item has one row
 ])
 def test_augment_small(case):
     wl = Workload("aug", case["grid"], case["heads"], 128, "bf16", 17, case["p"], case["k_min"],
