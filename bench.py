@@ -125,25 +125,40 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle arm (bounded sample of the same workload)
 # ---------------------------------------------------------------------------
-def oracle_sample(wl, q, k, v, budget_s: float, seed: int = 0):
-    """Time the oracle as it stands on a bounded sample: the coarse stage of
-    every head, then the fine stage of randomly drawn (head, query tile)
-    rows until the budget is spent.  Returns (est_full_seconds, flops_full,
-    description, threads)."""
+def oracle_sample(wl, q, k, v, budget_s: float, seed: int = 0, gpu_lists=None):
+    """Time the oracle as it stands on a bounded sample: the coarse stage
+    (pool, scores, top-p selection) head by head, then the fine stage of
+    randomly drawn (head, query tile) rows until the budget is spent.  With
+    ``gpu_lists`` = (counts, idx) host arrays [B, H, nT(, cap)] the coarse
+    stage runs on every head and each head's GPU lists are checked against
+    the oracle's (oracle/list_check.py) on every row.
+
+    Returns a dict: est_s (the whole workload, scaled by heads and by
+    selected pairs), flops, stage_s (coarse: measured, scaled by heads;
+    fine: scaled by selected pairs), desc, threads, and parity (or None)."""
     from oracle import fvattn_oracle as O
+    from oracle.list_check import check_lists, merge
     rope = dict(dims=wl.rope_dims, base=wl.rope_base) if wl.rope else None
     pos = O.positions(wl.grid, wl.order)
     scale = O.default_scale(wl.head_dim)
     t0 = time.perf_counter()
     coarse = []
     coarse_heads = 0
+    parity = None
+    t_check = 0.0
     for h in range(wl.heads):
         coarse.append(O.coarse_head(O.as_f64(q[0, h], wl.dtype), O.as_f64(k[0, h], wl.dtype), wl.grid, wl.order,
                                     wl.top_p, wl.k_min, scale, rope, pos))
         coarse_heads += 1
-        if time.perf_counter() - t0 > budget_s / 2 and h < wl.heads - 1:
+        if gpu_lists is not None:
+            tc = time.perf_counter()
+            one = check_lists(coarse[-1], gpu_lists[0][0, h], gpu_lists[1][0, h], wl.top_p, wl.k_min)
+            one["bad_rows"] = [(h, r) for r in one["bad_rows"]]
+            parity = merge(parity or {}, one)
+            t_check += time.perf_counter() - tc
+        elif time.perf_counter() - t0 > budget_s / 2 and h < wl.heads - 1:
             break
-    t_coarse = time.perf_counter() - t0
+    t_coarse = time.perf_counter() - t0 - t_check
     pairs_per_head = [int(r["counts"].sum()) for r in coarse]
     est_pairs_total = sum(pairs_per_head) * wl.heads / coarse_heads
     rng = np.random.default_rng(seed)
@@ -165,12 +180,13 @@ def oracle_sample(wl, q, k, v, budget_s: float, seed: int = 0):
         done_pairs += int(r["counts"][i])
         rows += 1
     t_fine = time.perf_counter() - t1
-    est = t_coarse * wl.heads / coarse_heads + t_fine * est_pairs_total / max(done_pairs, 1)
+    coarse_s = t_coarse * wl.heads / coarse_heads
+    fine_s = t_fine * est_pairs_total / max(done_pairs, 1)
     desc = (f"oracle (numpy fp64) coarse stage of {coarse_heads}/{wl.heads} heads + fine stage of {rows} random "
             f"(head, query tile) rows ({done_pairs} selected pairs of ~{int(est_pairs_total)}), scaled to the full "
             f"workload by heads and by selected pairs")
-    flops = est_pairs_total * pair_flops(wl.head_dim)
-    return est, flops, desc, _threads()
+    return dict(est_s=coarse_s + fine_s, flops=est_pairs_total * pair_flops(wl.head_dim),
+                stage_s={"coarse": coarse_s, "fine": fine_s}, desc=desc, threads=_threads(), parity=parity)
 
 
 def _threads():
@@ -183,6 +199,24 @@ def _threads():
         return os.cpu_count() or 1
 
 
+def workload_config(wl, args, world: int = 1) -> dict:
+    """The workload as both arms name it (no measured figures)."""
+    qk_bytes = 2 * wl.heads * wl.tokens * wl.head_dim * 2
+    return {"workload": wl.name, "grid": list(wl.grid), "tokens": wl.tokens, "heads": wl.heads,
+            "head_dim": wl.head_dim, "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order, "rope": wl.rope,
+            "scoring": "sub-block 2x2x2" if getattr(args, "subblock", False) else "tile mean",
+            "l2": "inputs larger than L2 (q+k+v = %.0f MB)" % (3 * qk_bytes / 2 / 1e6),
+            "parallelism": f"replica x{world}"}
+
+
+def cpu_baseline_of(res: dict) -> dict:
+    return {"value": res["flops"] / res["est_s"] / 1e12, "unit": UNIT, "cores": res["threads"],
+            "nproc": os.cpu_count(), "kind": "oracle", "sample": res["desc"],
+            "est_ms_per_step": res["est_s"] * 1e3,
+            "stage_ms": {k: v * 1e3 for k, v in res["stage_s"].items()},
+            "ms_is": "estimate: the sample's time scaled to the whole workload"}
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -191,19 +225,20 @@ def run_reference(args, wl):
     per_step = max(0.5, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(wl, q, k, v, min(per_step, 2.0), seed=1)
-    secs, flops = [], None
-    desc, cores = "", 1
+    secs, res = [], None
     for s in range(args.steps):
-        est, flops, desc, cores = oracle_sample(wl, q, k, v, per_step, seed=100 + s)
-        secs.append(est)
+        res = oracle_sample(wl, q, k, v, per_step, seed=100 + s)
+        secs.append(res["est_s"])
     ms = 1000.0 * statistics.mean(secs)
-    value = flops / (ms / 1000.0) / 1e12
+    value = res["flops"] / (ms / 1000.0) / 1e12
+    desc, cores = res["desc"], res["threads"]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "ms_per_step_is": "an estimate: each step times the oracle on a bounded sample of the workload "
+                              "(about %.1f s of CPU work) and scales it to the whole workload" % per_step,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "grid": list(wl.grid), "heads": wl.heads, "head_dim": wl.head_dim,
-                       "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "config": workload_config(wl, args, int(os.environ.get("WORLD_SIZE", "1"))),
+            "cpu_baseline": dict(cpu_baseline_of(res), value=value),
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -367,13 +402,9 @@ def run_gpu(args, wl):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "grid": list(wl.grid), "tokens": wl.tokens, "heads": wl.heads,
-                       "head_dim": wl.head_dim, "top_p": wl.top_p, "k_min": wl.k_min, "order": wl.order,
-                       "rope": wl.rope, "selected_pairs": pairs,
-                       "scoring": "sub-block 2x2x2" if args.subblock else "tile mean",
-                       "density": pairs / (wl.heads * wl.num_tiles ** 2),
-                       "l2": "inputs larger than L2 (q+k+v = %.0f MB)" % (3 * qk_bytes / 2 / 1e6),
-                       "parallelism": f"replica x{world}"},
+            "config": workload_config(wl, args, world),
+            "selected_pairs": pairs,
+            "density": pairs / (wl.heads * wl.num_tiles ** 2),
             "stage_ms": stage_ms,
             "pool_select": {"ms": pool_select_ms, "gbs": qk_bytes / (pool_select_ms / 1e3) / 1e9,
                             "frac_of_hbm": qk_bytes / (pool_select_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
@@ -392,9 +423,14 @@ def run_gpu(args, wl):
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
-            est, flops, desc, cores = oracle_sample(wl, q, k, v, budget_s=args.cpu_budget)
-            line["cpu_baseline"] = {"value": flops / est / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                    "sample": desc, "est_ms_per_step": est * 1e3}
+            # the oracle leg: its coarse stage runs on every head and checks the GPU's lists row by row
+            lists = None if args.subblock else (counts.cpu().numpy(), idx.cpu().numpy())
+            res = oracle_sample(wl, q, k, v, budget_s=args.cpu_budget, gpu_lists=lists)
+            line["cpu_baseline"] = cpu_baseline_of(res)
+            if res["parity"] is not None:
+                line["parity"] = dict(res["parity"], what="block lists of the timed forward vs the oracle, every "
+                                      "row of every head; borderline / near-tie rows that differ must be valid "
+                                      "lists")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -51,11 +51,19 @@ namespace ft {
 #ifndef FVATTN_FT_QBUF
 #define FVATTN_FT_QBUF 1
 #endif
+// MMA issue: 0 = lane 0 of warps 1 (S) and 2 (PV); 1 = the same two roles as
+// whole warps with an elected issuing lane; 2 = one warp issues both, PV(c)
+// then S(c + 2), so S never waits for a PV to complete (in-order execution
+// of one thread's tcgen05.mma keeps S(c + 2) from overwriting P(c) early).
+#ifndef FVATTN_FT_ISSUE
+#define FVATTN_FT_ISSUE 0
+#endif
 constexpr int D = 128;
 constexpr int KST = FVATTN_FT_KSTAGES;     // K ring depth
 constexpr int VST = FVATTN_FT_VSTAGES;     // V ring depth
 constexpr int QBUF = FVATTN_FT_QBUF;       // Q buffers (items in flight)
 constexpr int SBUF = 2;                    // TMEM S buffers
+constexpr int ISSUE = FVATTN_FT_ISSUE;
 constexpr int THREADS = 384;
 constexpr int SM_WARP0 = 4;                             // first softmax warp
 constexpr uint32_t BOX = 64 * 128;                      // one 64-row x 128-byte box: 8 KB
@@ -265,6 +273,32 @@ __device__ inline void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
       : "memory");
 }
 
+// S = Q K^T of one step (M=128 rows, N=128 keys, K=128 dims in 8 MMAs of
+// K=16) into TMEM at tS; Q and K in 128-byte swizzled d-halves.
+__device__ __forceinline__ void s_mmas(uint32_t tS, uint64_t qd, uint64_t kd) {
+  using namespace ft;
+  mma_ss(tS, qd, kd, IDESC_S, 0u);
+#pragma unroll
+  for (int kk = 1; kk < 8; ++kk)
+    mma_ss(tS, qd + (((kk >> 2) * Q_HALF + (kk & 3) * 32) >> 4), kd + (((kk >> 2) * K_HALF + (kk & 3) * 32) >> 4),
+           IDESC_S, 1u);
+}
+
+// O_t (+)= P_t V_t for the step's key tiles t = 0, 1: P_t (bf16) in TMEM at
+// tP + 64 t, V_t MN-major in the stage; 16 keys = 16 V rows = 2048 bytes
+// per K=16 MMA.
+__device__ __forceinline__ void pv_mmas(uint32_t tbase, uint32_t tP, const uint8_t* vstage, bool first) {
+  using namespace ft;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const uint64_t vd = umma_desc_sw128(smem_u32(vstage + t * V_TILE), BOX, 1024);
+    const uint32_t tO = tbase + TMEM_O + 128 * t;
+    mma_ts(tO, tP + 64 * t, vd, IDESC_PV, first ? 0u : 1u);
+#pragma unroll
+    for (int kk = 1; kk < 4; ++kk) mma_ts(tO, tP + 64 * t + 8 * kk, vd + ((kk * 2048) >> 4), IDESC_PV, 1u);
+  }
+}
+
 __global__ void __launch_bounds__(ft::THREADS, 1)
     fine_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, const FineTcArgs a) {
@@ -302,7 +336,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     mbar_init(&ctl->o_empty, 256);
     mbar_init(&ctl->xchg1, 128);
     mbar_init(&ctl->xchg2, 128);
-    mbar_init(&ctl->drain, 2);           // one final commit per MMA thread
+    mbar_init(&ctl->drain, ISSUE == 2 ? 1 : 2);   // one final commit per MMA issuer
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -417,7 +451,153 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         mbar_drain(&ctl->v_full[i], (uint32_t)(last / VST) & 1, a.status, cap);
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (ISSUE == 1 && warp == 1) {
+    // ------------------------------------------- MMA: S (whole warp, elected lane)
+    long long c = 0;
+    int k = 0;
+    bool ok = true;
+    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+      const int qb = k % QBUF;
+      if (!mbar_wait_warp(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
+      const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
+      while (true) {
+        const int ks = (int)(c % KST);
+        const int b = (int)(c & 1);
+        if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(c / KST) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        if (c >= SBUF &&
+            !mbar_wait_warp(&ctl->pv_done[b], (uint32_t)((c - SBUF) >> 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        const int meta = ctl->meta[ks];
+        tc_fence_after();
+        if (elect_one()) {
+          ctl->info[b] = meta;
+          s_mmas(tbase + 128 * b, qd, umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024));
+          mma_commit(&ctl->s_full[b]);
+          mma_commit(&ctl->k_empty[ks]);
+          if (meta & STEP_LAST) mma_commit(&ctl->q_empty[qb]);
+          mbar_arrive(&ctl->s_full[b]);
+        }
+        __syncwarp();
+        ++c;
+        if (meta & STEP_LAST) break;
+      }
+    }
+    if (elect_one()) mma_commit(&ctl->drain);
+    __syncwarp();
+    mbar_drain(&ctl->drain, 0, a.status, cap);
+  } else if (ISSUE == 1 && warp == 2) {
+    // ------------------------------------------ MMA: PV (whole warp, elected lane)
+    long long c = 0;
+    int k = 0;
+    bool ok = true;
+    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+      bool first = true;
+      while (true) {
+        const int b = (int)(c & 1);
+        const int vs = (int)(c % VST);
+        if (first && k >= 1 && !mbar_wait_warp(&ctl->o_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_warp(&ctl->v_full[vs], (uint32_t)(c / VST) & 1, abort_flag, a.status, cap) ||
+            !mbar_wait_warp(&ctl->p_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        const int info = ctl->info[b];
+        tc_fence_after();
+        if (elect_one()) {
+          pv_mmas(tbase, tbase + 128 * b, sV + vs * STAGE_BYTES, first);
+          mma_commit(&ctl->pv_done[b]);
+          mma_commit(&ctl->v_empty[vs]);
+        }
+        __syncwarp();
+        first = false;
+        ++c;
+        if (info & STEP_LAST) break;
+      }
+    }
+    if (elect_one()) mma_commit(&ctl->drain);
+    __syncwarp();
+    mbar_drain(&ctl->drain, 0, a.status, cap);
+  } else if (ISSUE == 2 && warp == 1) {
+    // ------------------------------------ MMA: S and PV from one warp, in order
+    // Order of issue: S(0), S(1), then per step c: PV(c) once P(c) is
+    // written, then S(c + 2) into the buffer PV(c) reads.  One thread's
+    // tcgen05.mma run in issue order, so S(c + 2) cannot overwrite P(c)
+    // before PV(c) has read it and S never waits for a PV to complete.
+    long long cs = 0, cp = 0;         // next S step, next PV step
+    int ks_item = 0, kp_item = 0;     // their items (in this CTA's slot order)
+    bool s_first = true, s_done = (int)blockIdx.x >= a.n_items, p_first = true;
+    int qb_s = 0;
+    uint64_t qd = 0;
+    auto issue_s = [&]() -> bool {
+      if (s_done) return true;
+      if (s_first) {
+        qb_s = ks_item % QBUF;
+        if (!mbar_wait_warp(&ctl->q_full[qb_s], (uint32_t)(ks_item / QBUF) & 1, abort_flag, a.status, cap))
+          return false;
+        qd = umma_desc_sw128(smem_u32(sQ + qb_s * Q_BYTES), 16, 1024);
+        s_first = false;
+      }
+      const int ks = (int)(cs % KST);
+      const int b = (int)(cs & 1);
+      if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(cs / KST) & 1, abort_flag, a.status, cap)) return false;
+      const int meta = ctl->meta[ks];
+      tc_fence_after();
+      if (elect_one()) {
+        ctl->info[b] = meta;
+        s_mmas(tbase + 128 * b, qd, umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024));
+        mma_commit(&ctl->s_full[b]);
+        mma_commit(&ctl->k_empty[ks]);
+        if (meta & STEP_LAST) mma_commit(&ctl->q_empty[qb_s]);
+        mbar_arrive(&ctl->s_full[b]);
+      }
+      __syncwarp();
+      ++cs;
+      if (meta & STEP_LAST) {
+        ++ks_item;
+        s_first = true;
+        if ((long long)blockIdx.x + (long long)ks_item * gridDim.x >= a.n_items) s_done = true;
+      }
+      return true;
+    };
+    bool ok = issue_s() && issue_s();
+    for (int slot = blockIdx.x; ok && slot < a.n_items;) {
+      const int b = (int)(cp & 1);
+      const int vs = (int)(cp % VST);
+      if (p_first && kp_item >= 1 &&
+          !mbar_wait_warp(&ctl->o_empty, (uint32_t)(kp_item - 1) & 1, abort_flag, a.status, cap))
+        break;
+      if (!mbar_wait_warp(&ctl->v_full[vs], (uint32_t)(cp / VST) & 1, abort_flag, a.status, cap) ||
+          !mbar_wait_warp(&ctl->p_full[b], (uint32_t)(cp >> 1) & 1, abort_flag, a.status, cap))
+        break;
+      const int info = ctl->info[b];
+      tc_fence_after();
+      if (elect_one()) {
+        pv_mmas(tbase, tbase + 128 * b, sV + vs * STAGE_BYTES, p_first);
+        mma_commit(&ctl->pv_done[b]);
+        mma_commit(&ctl->v_empty[vs]);
+      }
+      __syncwarp();
+      p_first = false;
+      ++cp;
+      if (info & STEP_LAST) {
+        ++kp_item;
+        p_first = true;
+        slot += gridDim.x;
+      }
+      ok = issue_s();
+    }
+    if (elect_one()) mma_commit(&ctl->drain);
+    __syncwarp();
+    mbar_drain(&ctl->drain, 0, a.status, cap);
+  } else if (ISSUE == 0 && warp == 1 && lane == 0) {
     // ------------------------------------------------------------- MMA: S
     // S(c) into buffer c & 1 once the PV of step c - 2, which read its P
     // from that buffer, is complete; a K stage is released when its S
@@ -463,7 +643,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     // every MMA this thread issued has completed before TMEM is freed
     mma_commit(&ctl->drain);
     mbar_drain(&ctl->drain, 0, a.status, cap);
-  } else if (warp == 2 && lane == 0) {
+  } else if (ISSUE == 0 && warp == 2 && lane == 0) {
     // ------------------------------------------------------------ MMA: PV
     // O_t += P_t V_t for the step's key tiles t = 0, 1 once both softmax
     // groups wrote P; the first step of an item overwrites O after the

@@ -298,6 +298,25 @@ __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* a
   }
 }
 
+// One lane of a converged warp returns true (elect.sync over the full mask).
+// Issuing tcgen05 work from an elected lane inside warp-uniform control flow
+// keeps descriptors and TMEM addresses warp-uniform.
+__device__ inline bool elect_one() {
+  uint32_t p = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b32 L;\n\telect.sync L|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
+// mbar_wait by every lane of a converged warp; the result is lane 0's, so
+// the warp leaves the wait together.
+__device__ inline bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                      long long cap) {
+  const bool ok = mbar_wait(bar, parity, abort, status, cap);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // Wait that ignores `abort`: used on the way out to let copies or MMAs that
 // were already issued land before the block exits or frees TMEM.
 __device__ inline bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, long long cap) {

@@ -20,8 +20,10 @@
 
 // 32 MiB.  A shape is accepted when its full workspace
 // (fvattn_workspace_size) fits: for example the 16x32x32 latent with 12
-// heads (7.6 MiB) or the 20x32x52 latent with up to 8 heads (16.6 MiB); the
-// 20x32x52 latent with 40 heads (82.5 MiB) is rejected.
+// heads (13.6 MiB) or the 20x32x52 latent with up to 8 heads (28.9 MiB); the
+// 20x32x52 latent with 9 heads (32.5 MiB) or 40 heads (144.1 MiB) is
+// rejected.  The first 4 bytes hold the status word that kernels set on a
+// device-detected error (fvattn_pool_select_noalloc_status reads it).
 static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 
 static __device__ __align__(256) unsigned char g_pool_select_scratch[kNoAllocScratchBytes];
@@ -58,4 +60,18 @@ extern "C" int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void*
   const int sa = scratch_address(&scratch);
   if (sa != FVATTN_OK) return sa;
   return fvattn_pool_select(shape, q, k, rope, top_p, k_min, out, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" int fvattn_pool_select_noalloc_status(fvattn_stream_t stream, int32_t* status) {
+  if (!status) return FVATTN_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const int sa = scratch_address(&scratch);
+  if (sa != FVATTN_OK) return sa;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FVATTN_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FVATTN_ERR_CUDA;
+  if (cudaMemset(scratch, 0, sizeof(v)) != cudaSuccess) return FVATTN_ERR_CUDA;
+  *status = v;
+  return FVATTN_OK;
 }

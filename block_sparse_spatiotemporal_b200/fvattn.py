@@ -22,7 +22,7 @@ __all__ = [
     "pool_select_subblock",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
-    "STAGES", "pool_select_noalloc", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
+    "STAGES", "pool_select_noalloc", "noalloc_status", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
     "augment_lists", "block_sparse_fwd_worklist", "timestep_params",
 ]
 
@@ -88,6 +88,7 @@ _SIGS = {
                                     ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_pool_select_noalloc": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
                                    ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p],
+    "fvattn_pool_select_noalloc_status": [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)],
     "fvattn_build_worklist": [ctypes.POINTER(Shape), ctypes.POINTER(Blocks), ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_block_sparse_fwd": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -267,6 +268,15 @@ def pool_select_noalloc(shape: Shape, q, k, top_p: float, k_min: int, rope: Opti
            lib().fvattn_pool_select_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope), float(top_p),
                                             int(k_min), ctypes.byref(b), _stream(stream)))
     return counts, idx
+
+
+def noalloc_status(stream=None) -> int:
+    """Read and clear the device status word of pool_select_noalloc
+    (synchronises the stream)."""
+    v = ctypes.c_int32(0)
+    _check("fvattn_pool_select_noalloc_status", lib().fvattn_pool_select_noalloc_status(_stream(stream),
+                                                                                       ctypes.byref(v)))
+    return int(v.value)
 
 
 def _blocks_of(counts, idx):

@@ -173,6 +173,18 @@ int fvattn_pool_select_noalloc(const fvattn_shape* shape, const void* q, const v
                                const fvattn_rope* rope, float top_p, int32_t k_min,
                                const fvattn_blocks* out, fvattn_stream_t stream);
 
+/* Device status of fvattn_pool_select_noalloc (the pages have no
+ * counterpart either).  A caller without a workspace cannot pass one to
+ * fvattn_get_device_status, so this reads the status word that the
+ * kernels of fvattn_pool_select_noalloc set on a device-detected error (0:
+ * none; 1: an out-of-range block index; 2: a wait that hit its iteration
+ * cap) from the library's own scratch array, clears it, and returns it in
+ * *status (a HOST pointer).  It synchronises `stream` first, then copies
+ * 4 bytes with cudaMemcpy; it allocates nothing.  Call it on the device
+ * and stream of the noalloc calls it checks; calls that overlap race as
+ * above. */
+int fvattn_pool_select_noalloc_status(fvattn_stream_t stream, int32_t* status);
+
 /* Schedule of the fine stage (single-GPU analogue of the "FVAttn" digest's
  * runtime head-level load balancing, section 02): a work item is two
  * adjacent query tiles 2q, 2q+1 of one (batch, head), encoded

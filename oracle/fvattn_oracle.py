@@ -33,7 +33,7 @@ Sources (page title, section):
     index t + s of a block starting at frame s, and the QKV projection fused
     with the rotation.
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
   * pooling is the mean over the 64 tokens of a tile;
   * coarse logits are scale * Qp . Kp with scale = 1/sqrt(d); normalisation is
     a softmax over the key tiles of each query-tile row;
@@ -72,8 +72,8 @@ Readings where the pages are silent (each also listed in the design notes):
     section 2.2), V is not; the results are rounded once to bf16.
 
 Every function below is pinned by ``tests/test_oracle_*.py`` against brute
-force, closed forms, invariants or library routines; see the pin list in the
-design notes.
+force, closed forms, invariants or library routines; each test's docstring
+names what it pins.
 """
 from __future__ import annotations
 

@@ -9,6 +9,7 @@ import torch
 from block_sparse_spatiotemporal_b200 import fvattn as F
 from block_sparse_spatiotemporal_b200.inputs import Workload
 from oracle import fvattn_oracle as O
+from oracle.list_check import check_lists, merge
 
 BF16_MAX_ABS, BF16_MEAN_ABS = 2e-2, 2e-3
 F32_ABS = 1e-4
@@ -48,40 +49,29 @@ def oracle_coarse(wl: Workload, q, k, top_p, k_min, b=0, heads=None):
     return out
 
 
-def compare_blocks(res: dict, gpu_counts: np.ndarray, gpu_idx: np.ndarray, top_p: float):
-    """Compare one head's GPU lists with the oracle's.
+def compare_blocks(res: dict, gpu_counts: np.ndarray, gpu_idx: np.ndarray, top_p: float, k_min: int):
+    """Compare one head's GPU lists with the oracle's (oracle/list_check.py).
 
-    Returns (n_mismatch, n_border, n_neartie_checked, equal_rows).  Rows whose
-    cumulative mass lies within 1e-5 of top_p at the cut are exempt (counted).
-    Near-tie rows -- the last kept and first dropped logits closer than the
-    float32 rounding bound of a 128-term dot product (1e-5 of the row's
-    largest scale * |Qp|.|Kp|) -- may select either tile, but the GPU set must
-    still be a top-count set within that bound.  Any other difference is a
-    mismatch."""
-    S, counts, idx, border = res["S"], res["counts"], res["idx"], res["border"]
-    nT = S.shape[0]
-    tol = 1e-5 * res["s_abs"].max(axis=1)
-    near = O.near_tie_rows(S, counts, tol)
-    mism = 0
-    ntie = 0
-    equal = np.zeros(nT, bool)
-    for r in range(nT):
-        c = int(gpu_counts[r])
-        same = c == counts[r] and np.array_equal(gpu_idx[r, :c], idx[r, :counts[r]])
-        equal[r] = same
-        if same or border[r]:
-            continue
-        if near[r] and c == counts[r]:
-            sel = gpu_idx[r, :c]
-            ok = len(set(sel.tolist())) == c and (np.diff(sel) > 0).all()
-            rest = np.setdiff1d(np.arange(nT), sel)
-            if ok and len(rest):
-                ok = S[r, sel].min() >= S[r, rest].max() - tol[r]
-            ntie += 1
-            if ok:
-                continue
-        mism += 1
-    return mism, int(border.sum()), ntie, equal
+    Returns the checker's row counts plus ``equal_rows`` (bool per row).
+    Borderline rows (cumulative mass within 1e-5 of top_p at the cut) and
+    near-tie rows (last kept and first dropped logits within the float32
+    rounding bound) may differ from the oracle's list but must be valid:
+    ids ascending and in range, the count between the counts at
+    top_p -/+ 1e-5 (borderline) or equal to the oracle's (near tie), and a
+    top-count set of the row's logits up to the rounding bound.  Any other
+    difference is a mismatch."""
+    equal = np.zeros(len(gpu_counts), bool)
+    out = check_lists(res, gpu_counts, gpu_idx, top_p, k_min, equal_rows=equal)
+    out["equal_rows"] = equal
+    return out
+
+
+def sum_checks(checks):
+    """Row counts of several heads' compare_blocks results, summed."""
+    tot = {}
+    for c in checks:
+        merge(tot, {k: v for k, v in c.items() if k != "equal_rows"})
+    return tot
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str):

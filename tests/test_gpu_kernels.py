@@ -11,7 +11,7 @@ import torch
 from block_sparse_spatiotemporal_b200 import fvattn as F
 from block_sparse_spatiotemporal_b200.inputs import Workload, WORKLOADS, make_inputs
 from oracle import fvattn_oracle as O
-from tests.gpu_util import (assert_close, compare_blocks, oracle_coarse, oracle_rope, rope_of, shape_of,
+from tests.gpu_util import (assert_close, compare_blocks, sum_checks, oracle_coarse, oracle_rope, rope_of, shape_of,
                             to_dev, to_host)
 
 pytestmark = pytest.mark.gpu
@@ -69,11 +69,8 @@ def _pool_select_case(wl, layout=F.NATURAL, top_p=None, k_min=None):
     assert F.device_status(ws) == 0
     gc, gi = _blocks_host(counts, idx)
     res = oracle_coarse(wl, q, k, top_p, k_min)
-    total_mism = 0
-    for h, r in enumerate(res):
-        mism, _, _, _ = compare_blocks(r, gc[0, h], gi[0, h], top_p)
-        total_mism += mism
-    assert total_mism == 0
+    tot = sum_checks([compare_blocks(r, gc[0, h], gi[0, h], top_p, k_min) for h, r in enumerate(res)])
+    assert tot["mismatch"] == 0, tot
     return q, k, v, res, gc, gi
 
 

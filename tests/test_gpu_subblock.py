@@ -7,7 +7,7 @@ import pytest
 from block_sparse_spatiotemporal_b200 import fvattn as F
 from block_sparse_spatiotemporal_b200.inputs import Workload, WORKLOADS, make_inputs
 from oracle import fvattn_oracle as O
-from tests.gpu_util import assert_close, compare_blocks, oracle_rope, rope_of, shape_of, to_dev, to_host
+from tests.gpu_util import assert_close, compare_blocks, sum_checks, oracle_rope, rope_of, shape_of, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -43,10 +43,9 @@ def run_sub(wl, top_p, k_min, layout=F.NATURAL, heads=None):
     assert F.device_status(ws) == 0
     gc, gi = counts.cpu().numpy(), idx.cpu().numpy()
     res = oracle_sub(wl, q, k, top_p, k_min, heads)
-    mism = border = ties = 0
-    for n, h in enumerate(range(wl.heads) if heads is None else heads):
-        m, b, t, _ = compare_blocks(res[n], gc[0, h], gi[0, h], top_p)
-        mism, border, ties = mism + m, border + b, ties + t
+    tot = sum_checks([compare_blocks(res[n], gc[0, h], gi[0, h], top_p, k_min)
+                      for n, h in enumerate(range(wl.heads) if heads is None else heads)])
+    mism, border, ties = tot["mismatch"], tot["borderline"], tot["near_tie"]
     return dict(q=q, k=k, v=v, shape=shape, rope=rope, ws=ws, counts=counts, idx=idx, gc=gc, gi=gi, res=res,
                 mism=mism, border=border, ties=ties)
 
