@@ -171,9 +171,8 @@ def oracle_sample(wl, q, k, v, budget_s: float, seed: int = 0, gpu_lists=None):
         i = int(rng.integers(wl.num_tiles))
         r = coarse[h]
         if h not in vt_cache:
-            qt, kt = r["q_tiled"], r["k_tiled"]
-            if wl.rope and wl.dtype == "bf16":
-                qt, kt = O.round_bf16(qt), O.round_bf16(kt)
+            qt, kt = O.fine_operands(O.as_f64(q[0, h], wl.dtype), O.as_f64(k[0, h], wl.dtype), wl.grid, wl.dtype,
+                                     rope, pos)
             vt_cache = {h: (qt, kt, O.to_tiled(O.as_f64(v[0, h], wl.dtype), pos))}
         qt, kt, vt = vt_cache[h]
         O.fine_tile(qt[i * 64:(i + 1) * 64], kt, vt, r["idx"][i, :r["counts"][i]], scale)

@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "order.cu", "coarse.cu", "scores_tc.cu", "subblock.cu", "schedule.cu", "fine_tc.cu", "fine_f32.cu", "qkv_tc.cu", "bwd_tc.cu", "augment.cu", "selftest.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "order.cu", "coarse.cu", "scores_tc.cu", "subblock.cu", "schedule.cu", "fine_tc.cu", "fine_q.cu", "fine_f32.cu", "qkv_tc.cu", "bwd_tc.cu", "augment.cu", "selftest.cu", "noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "fvattn_internal.cuh"), os.path.join(ROOT, "include", "fvattn.h")]
 LIB = os.path.join(HERE, "libfvattn.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -62,6 +62,7 @@ int make_geom(const fvattn_shape* s, Geom* g) {
   g->N = (int)N;
   g->BH = (int)BH;
   g->P = (int)((nT + kItemTiles - 1) / kItemTiles);
+  g->Qn = (int)((nT + 3) / 4);
   g->order = s->order;
   g->scale = s->scale > 0.f ? s->scale : (float)(1.0 / std::sqrt((double)d));
   return FVATTN_OK;
@@ -105,6 +106,8 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   L.ucount = take(sizeof(int) * (size_t)g.BH * g.P);
   L.worklist = take(sizeof(int) * (size_t)g.BH * g.P);
   L.rank = take(sizeof(int) * (size_t)g.BH * g.P);
+  L.useg = take(sizeof(int) * (size_t)g.BH * g.Qn);
+  L.qcost = take(sizeof(int) * (size_t)g.BH * g.Qn);
   const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
   L.qrot = take(rot);
   L.krot = take(rot);
@@ -423,8 +426,26 @@ int run_schedule(const Call& c, const fvattn_blocks* blocks, int* worklist) {
   StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
   FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
                        c.status, c.s));
-  FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, c.at<int>(c.L.rank), worklist, c.s));
-  t.kernels = 3;      // union, partial ranks, scatter
+  FV_CUDA(launch_rank(c.at<int>(c.L.ucount), c.g.BH * c.g.P, c.g.nT, worklist, c.s));
+  t.kernels = 2;      // union, counting sort
+  return FVATTN_OK;
+}
+
+// Fine-stage kernel of the forward: 1 = quad items (fine_q_kernel, four
+// query tiles sharing one K/V stream), 0 = two-tile items (fine_tc_kernel).
+#ifndef FVATTN_FINE_QUAD
+#define FVATTN_FINE_QUAD 0
+#endif
+constexpr bool kFineQuad = FVATTN_FINE_QUAD != 0;
+
+// Schedule of the quad items of the forward's fine stage: union lists in
+// the order both halves / A only / B only, and the longest-first work list.
+int run_schedule_quad(const Call& c, const fvattn_blocks* blocks) {
+  StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
+  FV_CUDA(launch_quad_schedule(c.g, c.g.Qn, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni),
+                               c.at<int>(c.L.ucount), c.at<int>(c.L.useg), c.at<int>(c.L.qcost),
+                               c.at<int>(c.L.worklist), c.status, c.s));
+  t.kernels = 2;      // quad unions, counting sort
   return FVATTN_OK;
 }
 
@@ -438,7 +459,34 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
   const void* qs = r ? c.at<void>(c.L.qrot) : q;
   const void* ks = r ? c.at<void>(c.L.krot) : k;
   const bool qk_nat = natural && !r;
-  if (shape->dtype == FVATTN_BF16) {
+  if (kFineQuad && shape->dtype == FVATTN_BF16 && !worklist) {
+    // quad items over the schedule of run_schedule_quad
+    CUtensorMap mq, mk, mv;
+    FV_TRY(make_tile_map(&mq, qs, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mk, ks, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mv, v, c.g, natural));
+    FineQArgs a{};
+    a.g = c.g;
+    a.uni = c.at<int>(c.L.uni);
+    a.ucount = c.at<int>(c.L.ucount);
+    a.useg = c.at<int>(c.L.useg);
+    a.worklist = c.at<int>(c.L.worklist);
+    a.n_items = c.g.BH * c.g.Qn;
+    a.Qn = c.g.Qn;
+    a.tile_cube = c.at<int>(c.L.tile_cube);
+    a.q_nat = qk_nat;
+    a.k_nat = qk_nat;
+    a.v_nat = natural;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.out_nat = natural;
+    a.status = c.status;
+    a.wait_cap = kDefaultWaitCap;
+    StageTimer t(FVATTN_STAGE_FINE, c.s);
+    FV_CUDA(launch_fine_q(mq, mk, mv, a, grid > 0 ? grid : c.dev.sms, c.s));
+    t.kernels = a.n_items > 0 ? 1 : 0;
+  } else if (shape->dtype == FVATTN_BF16) {
+    // two-tile items over a caller's work list (augmented lists)
     CUtensorMap mq, mk, mv;
     FV_TRY(make_tile_map(&mq, qs, c.g, qk_nat));
     FV_TRY(make_tile_map(&mk, ks, c.g, qk_nat));
@@ -608,7 +656,8 @@ int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
   if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
-  FV_TRY(run_schedule(c, blocks, c.at<int>(c.L.worklist)));
+  if (shape->dtype == FVATTN_BF16) FV_TRY(kFineQuad ? run_schedule_quad(c, blocks)
+                                                   : run_schedule(c, blocks, c.at<int>(c.L.worklist)));
   FV_TRY(run_fine(c, shape, q, k, v, rope, natural, blocks, out, lse));
   return FVATTN_OK;
 }
@@ -705,7 +754,8 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
   } else if (rope_on(rope)) {
     FV_TRY(run_coarse(c, &sh, q, k, rope, true, false, true, 0.f, 0, blocks));
   }
-  FV_TRY(run_schedule(c, blocks, c.at<int>(c.L.worklist)));
+  if (sh.dtype == FVATTN_BF16) FV_TRY(kFineQuad ? run_schedule_quad(c, blocks)
+                                               : run_schedule(c, blocks, c.at<int>(c.L.worklist)));
   FV_TRY(run_fine(c, &sh, q, k, v, rope, true, blocks, out, lse));
   if (cache && !reuse_mask) {
     cache->shape = sh;
@@ -741,11 +791,11 @@ int fvattn_block_sparse_bwd(const fvattn_shape* shape, const void* q, const void
     StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
     FV_CUDA(launch_union(g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
                          c.status, c.s));
-    FV_CUDA(launch_rank(c.at<int>(c.L.ucount), g.BH * g.P, c.at<int>(c.L.rank), c.at<int>(c.L.worklist), c.s));
+    FV_CUDA(launch_rank(c.at<int>(c.L.ucount), g.BH * g.P, g.nT, c.at<int>(c.L.worklist), c.s));
     FV_CUDA(launch_key_union(g, blocks->counts, blocks->idx, blocks->cap, c.at<uint32_t>(c.L.bits),
                              c.at<int>(c.L.uni_t), c.at<int>(c.L.ucount_t), c.status, c.s));
-    FV_CUDA(launch_rank(c.at<int>(c.L.ucount_t), g.BH * g.P, c.at<int>(c.L.rank_t), c.at<int>(c.L.worklist_t), c.s));
-    t.kernels = 7;   // union, 2 x (partial ranks, scatter), transpose bits, key union
+    FV_CUDA(launch_rank(c.at<int>(c.L.ucount_t), g.BH * g.P, g.nT, c.at<int>(c.L.worklist_t), c.s));
+    t.kernels = 5;   // union, 2 x counting sort, transpose bits, key union
   }
   CUtensorMap mq, mk, mv, mdo;
   FV_TRY(make_tile_map(&mq, q, g, false));

@@ -52,9 +52,12 @@ __device__ inline void rope_pair(const RopeArgs& r, const Geom& g, int dim, int 
   } else {
     cs = r.tab[g.T * (r.dt / 2) + g.Hg * (r.dh / 2) + w * (r.dw / 2) + (dim - r.dt - r.dh) / 2];
   }
+  // each product and the sum / difference rounded to float32 on its own (no
+  // fused multiply-add), so the values rounded to the operand dtype are
+  // reproducible: the oracle evaluates the same expression in float32
   const float x0 = a, x1 = b;
-  a = x0 * cs.x - x1 * cs.y;
-  b = x0 * cs.y + x1 * cs.x;
+  a = __fsub_rn(__fmul_rn(x0, cs.x), __fmul_rn(x1, cs.y));
+  b = __fadd_rn(__fmul_rn(x0, cs.y), __fmul_rn(x1, cs.x));
 }
 
 // --------------------------------------------------------------------------

@@ -36,7 +36,8 @@ struct Geom {
   int nT;                // tiles per head
   int N;                 // tokens per head
   int BH;
-  int P;                 // fine-stage work items per head = ceil(nT / kItemTiles)
+  int P;                 // two-tile work items per head = ceil(nT / kItemTiles)
+  int Qn;                // quad work items per head = ceil(nT / 4)
   int order;             // fvattn_order
   float scale;           // softmax scale
 };
@@ -54,6 +55,7 @@ struct WsLayout {
   size_t counts, idx;    // int32 [BH*nT], [BH*nT*nT] (forward without cache)
   size_t uni, ucount;    // int32 [BH*P*nT], [BH*P]
   size_t worklist;       // int32 [BH*P]
+  size_t useg, qcost;    // int32 [BH*Qn] quad items: union segments and cost
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
@@ -93,6 +95,24 @@ struct FineTcArgs {
   const int* ucount;
   const int* worklist;
   int n_items;
+  const int* tile_cube;
+  int q_nat, k_nat, v_nat;
+  __nv_bfloat16* out;
+  float* lse;
+  int out_nat;
+  int* status;
+  long long wait_cap;
+};
+
+// Fine stage over quad items (four query tiles in two 128-row halves).
+struct FineQArgs {
+  Geom g;
+  const int* uni;        // [items][nT] union entries (key tile | selection bits << 16)
+  const int* ucount;     // [items] entries
+  const int* useg;       // [items] entries of both halves | entries of half A only << 16
+  const int* worklist;   // [items] longest first
+  int n_items;
+  int Qn;                // quad items per (batch, head) = ceil(nT / 4)
   const int* tile_cube;
   int q_nat, k_nat, v_nat;
   __nv_bfloat16* out;
@@ -478,10 +498,16 @@ cudaError_t launch_scores_sub(const CUtensorMap& mqh, const CUtensorMap& mql, co
 cudaError_t launch_subblock_agg(const Geom& g, const float* Tb, float* logp, cudaStream_t s);
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
                          cudaStream_t s);
-cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s);
+// Longest-first order of n items by key (descending; ties by ascending item
+// index), keys in [0, max_key].
+cudaError_t launch_rank(const int* key, int n, int max_key, int* worklist, cudaStream_t s);
 cudaError_t launch_fine_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineTcArgs& a,
                            int num_sms, cudaStream_t s);
 cudaError_t launch_fine_f32(const FineF32Args& a, cudaStream_t s);
+cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const int* idx, int cap, int* uni,
+                                 int* ucount, int* useg, int* qcost, int* worklist, int* status, cudaStream_t s);
+cudaError_t launch_fine_q(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineQArgs& a,
+                          int num_sms, cudaStream_t s);
 cudaError_t launch_token_pos(const Geom& g, const int* cube_rank, int* pos, cudaStream_t s);
 cudaError_t launch_rope_pairs(const Geom& g, int dt, int dh, int dw, float base, int t_offset, float2* tab,
                               cudaStream_t s);

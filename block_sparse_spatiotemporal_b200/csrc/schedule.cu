@@ -7,7 +7,8 @@
 // lists; each entry records which of the two tiles selected it (the other
 // tile's rows are masked for it).  Items are ranked by union size, longest
 // first (LPT), ties by item code, so the persistent fine kernel hands the
-// heavy items out first and the light ones fill the tail.
+// heavy items out first and the light ones fill the tail; the ranking is a
+// counting sort on the cost (lpt_sort_kernel).
 #include "fvattn_internal.cuh"
 
 namespace fvattn {
@@ -77,32 +78,149 @@ __global__ void __launch_bounds__(128) union_kernel(Geom g, const int* __restric
   }
 }
 
-// rank(e) = #{e' : key(e') > key(e)} + #{e' < e : key(e') == key(e)};
-// worklist[rank(e)] = e.  The comparisons are split over segments of e'
-// (grid y) whose partial counts are added into rank[] (integer adds, so the
-// result does not depend on their order); a second kernel scatters.
-constexpr int kRankSeg = 1024;
-
-__global__ void __launch_bounds__(256) rank_partial_kernel(const int* __restrict__ key, int n, int* __restrict__ rank) {
-  __shared__ int ks[kRankSeg];
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  const int s0 = blockIdx.y * kRankSeg;
-  const int len = min(kRankSeg, n - s0);
-  for (int i = threadIdx.x; i < len; i += blockDim.x) ks[i] = key[s0 + i];
-  __syncthreads();
-  if (e >= n) return;
-  const int ke = key[e];
-  int c = 0;
-  for (int i = 0; i < len; ++i) {
-    const int kk = ks[i];
-    c += (kk > ke || (kk == ke && s0 + i < e)) ? 1 : 0;
+// ---------------------------------------------------------------------------
+// Quad items of the fine stage: query tiles 4u .. 4u+3 of one (batch, head),
+// two halves of two tiles (A = 4u, 4u+1; B = 4u+2, 4u+3), each half one
+// 128-row tensor-core tile.  The item walks the union of the four tiles'
+// lists once; both halves share its K/V tiles.  Entries are ordered: key
+// tiles selected by both halves, then by half A only, then by half B only
+// (ascending within each group), so that each half is active on a prefix
+// and, for B, a suffix of the item's steps (two entries per step) and idle
+// elsewhere.
+//   entry: bits 0-15 key tile id, bits 16-19 selected by tile 4u + i.
+//   ucount[item] = entries, useg[item] = n_both | n_a << 16,
+//   qcost[item] = active steps of A + active steps of B.
+// One warp per item; lists are validated as in union_kernel.
+// ---------------------------------------------------------------------------
+__host__ __device__ inline void quad_steps(int n, int nb, int na, int* sa, int* sb) {
+  const int steps = (n + 1) >> 1;
+  *sa = (nb + na + 1) >> 1;
+  const int pre = (nb + 1) >> 1;
+  int b = pre;
+  if (n - nb - na > 0) {
+    const int start = (nb + na) >> 1;
+    const int overlap = pre > start ? pre - start : 0;
+    b += steps - start - overlap;
   }
-  if (c) atomicAdd(&rank[e], c);
+  *sb = b;
 }
 
-__global__ void scatter_rank_kernel(const int* __restrict__ rank, int n, int* __restrict__ worklist) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e < n) worklist[rank[e]] = e;
+__global__ void __launch_bounds__(128) quad_union_kernel(Geom g, int Qn, const int* __restrict__ counts,
+                                                         const int* __restrict__ idx, int cap, int* __restrict__ uni,
+                                                         int* __restrict__ ucount, int* __restrict__ useg,
+                                                         int* __restrict__ qcost, int* status) {
+  extern __shared__ uint32_t bm[];  // per warp: 4 bitmaps of ceil(nT/32) words
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int words = (g.nT + 31) / 32;
+  uint32_t* bmw = bm + warp * 4 * words;
+  const long long item = (long long)blockIdx.x * 4 + warp;
+  if (item >= (long long)g.BH * Qn) return;
+  const int bh = (int)(item / Qn), u = (int)(item % Qn);
+  for (int w = lane; w < 4 * words; w += 32) bmw[w] = 0u;
+  __syncwarp();
+  for (int t = 0; t < 4; ++t) {
+    const int tile = 4 * u + t;
+    if (tile >= g.nT) break;
+    const size_t row = (size_t)bh * g.nT + tile;
+    int c = counts[row];
+    if (c < 0 || c > g.nT) {
+      if (lane == 0) set_status(status, kStatusBadBlock);
+      c = c < 0 ? 0 : g.nT;
+    }
+    const int* list = idx + row * (size_t)cap;
+    uint32_t* bmx = bmw + t * words;
+    for (int e = lane; e < c; e += 32) {
+      const int j = list[e];
+      const bool ok = j >= 0 && j < g.nT && (e == 0 || list[e - 1] < j);
+      if (!ok) {
+        set_status(status, kStatusBadBlock);
+        continue;
+      }
+      atomicOr(&bmx[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncwarp();
+  int* out = uni + item * (long long)g.nT;
+  int n = 0, seg[3] = {0, 0, 0};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int n0 = n;
+    for (int w = 0; w < words; ++w) {
+      const int j = w * 32 + lane;
+      uint32_t sel = 0;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) sel |= ((bmw[t * words + w] >> lane) & 1u) << t;
+      const bool a = (sel & 3u) != 0u, b = (sel & 12u) != 0u;
+      const bool take = pass == 0 ? (a && b) : pass == 1 ? (a && !b) : (b && !a);
+      const unsigned bal = __ballot_sync(0xffffffffu, take);
+      if (take) out[n + __popc(bal & ((1u << lane) - 1u))] = j | (int)(sel << 16);
+      n += __popc(bal);
+    }
+    seg[pass] = n - n0;
+  }
+  if (lane == 0) {
+    ucount[item] = n;
+    useg[item] = seg[0] | (seg[1] << 16);
+    int sa, sb;
+    quad_steps(n, seg[0], seg[1], &sa, &sb);
+    qcost[item] = sa + sb;
+  }
+}
+
+// Longest-first work list by a counting sort on the cost: bins of equal
+// cost in descending order, items inside a bin in ascending code (head-major,
+// so the CTAs that start together share a head's K/V in L2).  One block:
+// histogram, a descending exclusive scan by one warp, then one warp places
+// the items 32 at a time in code order (ranks among equal costs from
+// __match_any_sync), which keeps the order stable and deterministic.
+__global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ cost, int n, int maxc,
+                                                        int* __restrict__ worklist) {
+  extern __shared__ int hist[];  // maxc + 1 bins
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i <= maxc; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += blockDim.x) atomicAdd(&hist[min(max(cost[i], 0), maxc)], 1);
+  __syncthreads();
+  if (tid >= 32) return;
+  int run = 0;
+  for (int c0 = maxc; c0 >= 0; c0 -= 32) {
+    const int c = c0 - lane;
+    const int v = c >= 0 ? hist[c] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (c >= 0) hist[c] = run + x - v;
+    run += __shfl_sync(0xffffffffu, x, 31);
+  }
+  __syncwarp();
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    const bool valid = i < n;
+    const int c = valid ? min(max(cost[i], 0), maxc) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, c);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int base = valid ? hist[c] : 0;
+    __syncwarp();
+    if (valid) {
+      worklist[base + rank] = i;
+      if ((peers >> lane) == 1u) hist[c] = base + __popc(peers);   // the group's highest lane advances the bin
+    }
+    __syncwarp();
+  }
+}
+
+cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const int* idx, int cap, int* uni,
+                                 int* ucount, int* useg, int* qcost, int* worklist, int* status, cudaStream_t s) {
+  const long long items = (long long)g.BH * Qn;
+  if (items <= 0) return cudaSuccess;
+  const int words = (g.nT + 31) / 32;
+  quad_union_kernel<<<(unsigned)((items + 3) / 4), 128, (size_t)4 * 4 * words * sizeof(uint32_t), s>>>(
+      g, Qn, counts, idx, cap, uni, ucount, useg, qcost, status);
+  const int maxc = 2 * ((g.nT + 1) / 2) + 2;
+  lpt_sort_kernel<<<1, 1024, (size_t)(maxc + 1) * sizeof(int), s>>>(qcost, (int)items, maxc, worklist);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
@@ -114,12 +232,9 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
   return cudaGetLastError();
 }
 
-cudaError_t launch_rank(const int* key, int n, int* rank, int* worklist, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(rank, 0, sizeof(int) * (size_t)n, s);
-  if (e != cudaSuccess) return e;
-  dim3 grid((n + 255) / 256, (n + kRankSeg - 1) / kRankSeg);
-  rank_partial_kernel<<<grid, 256, 0, s>>>(key, n, rank);
-  scatter_rank_kernel<<<(n + 255) / 256, 256, 0, s>>>(rank, n, worklist);
+cudaError_t launch_rank(const int* key, int n, int max_key, int* worklist, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  lpt_sort_kernel<<<1, 1024, (size_t)(max_key + 1) * sizeof(int), s>>>(key, n, max_key, worklist);
   return cudaGetLastError();
 }
 

@@ -48,8 +48,10 @@ Readings where the pages are silent:
   * lse is the natural log of the softmax normaliser;
   * RoPE: per-axis groups of 44/42/42 head dims for (t, h, w), adjacent pairs
     (2j, 2j+1) inside each group, angle = pos * base^(-2j/d_axis); pooling uses
-    the rotated values unrounded, the fine stage uses them rounded to bf16
-    (the tensor-core operand precision of a bf16 workload);
+    the rotated values unrounded (float64 here), the fine stage uses them as
+    its tensor-core operands hold them: rotated in float32 and, for a bf16
+    workload, rounded to bf16 (the rounding is a quantisation, so it is taken
+    from the same float32 values as the kernel's, see ``rope_3d_f32``);
   * Hilbert order: Skilling's transposed-axes Hilbert index ("Programming the
     Hilbert curve", AIP Conf. Proc. 707, 2004) on the enclosing 2^k cube with
     axes (t, h, w), valid tokens ordered by index;
@@ -224,6 +226,48 @@ def rope_3d(x, coords, dims=(44, 42, 42), base=10000.0):
         y[:, off + 1:off + da:2] = x0 * s + x1 * c
         off += da
     return y
+
+
+def rope_3d_f32(x, coords, dims=(44, 42, 42), base=10000.0):
+    """The rotation of ``rope_3d`` evaluated in float32, the precision of the
+    values that become the fine stage's tensor-core operands: each (cos, sin)
+    entry is the float64 value of pos * base^(-2j/d_a) rounded to float32,
+    and each product and the sum or difference is rounded to float32 on its
+    own (numpy float32 arithmetic, no fused multiply-add).  Rounding these
+    values to bf16 is a quantisation; taking it from float32 values that the
+    kernel reproduces exactly makes the two sides round identically, where
+    float64 values would round differently whenever one sits within a float32
+    rounding error of a bf16 boundary.  Returns float32 [N, d]."""
+    assert sum(dims) == x.shape[-1]
+    xf = np.asarray(x, dtype=np.float32)
+    y = np.array(xf, copy=True)
+    off = 0
+    for axis, da in enumerate(dims):
+        j = np.arange(da // 2, dtype=np.float64)
+        theta = base ** (-2.0 * j / da)
+        ang = coords[:, axis:axis + 1].astype(np.float64) * theta[None, :]
+        c, s = np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+        x0, x1 = xf[:, off + 0:off + da:2], xf[:, off + 1:off + da:2]
+        y[:, off + 0:off + da:2] = (x0 * c) - (x1 * s)
+        y[:, off + 1:off + da:2] = (x0 * s) + (x1 * c)
+        off += da
+    return y
+
+
+def fine_operands(q, k, grid, dtype, rope=None, pos=None):
+    """Tiled q, k as the fine stage consumes them: the inputs as given
+    (float64 of the bf16 / float32 values), or with RoPE the float32
+    rotation of ``rope_3d_f32``, rounded to bf16 for bf16 workloads."""
+    if pos is None:
+        pos = positions(grid, "raster")
+    if rope is None:
+        return to_tiled(q, pos), to_tiled(k, pos)
+    coords = token_coords(grid)
+    qr = rope_3d_f32(q, coords, rope["dims"], rope["base"]).astype(np.float64)
+    kr = rope_3d_f32(k, coords, rope["dims"], rope["base"]).astype(np.float64)
+    if dtype == "bf16":
+        qr, kr = round_bf16(qr), round_bf16(kr)
+    return to_tiled(qr, pos), to_tiled(kr, pos)
 
 
 def round_bf16(x):
@@ -730,16 +774,9 @@ def forward_head(q, k, v, grid, order, top_p, k_min, dtype, scale=None,
     if blocks is None:
         res = coarse_head(qf, kf, grid, order, top_p, k_min, scale, rope, pos)
         counts, idx = res["counts"], res["idx"]
-        qt, kt = res["q_tiled"], res["k_tiled"]
     else:
         counts, idx = blocks
-        if rope is not None:
-            coords = token_coords(grid)
-            qf = rope_3d(qf, coords, rope["dims"], rope["base"])
-            kf = rope_3d(kf, coords, rope["dims"], rope["base"])
-        qt, kt = to_tiled(qf, pos), to_tiled(kf, pos)
-    if rope is not None and dtype == "bf16":
-        qt, kt = round_bf16(qt), round_bf16(kt)
+    qt, kt = fine_operands(qf, kf, grid, dtype, rope, pos)
     vt = to_tiled(vf, pos)
     out_t, lse_t = fine_head(qt, kt, vt, counts, idx, scale, rows)
     res.update(out=from_tiled(out_t, pos), lse=lse_t[pos], out_tiled=out_t,

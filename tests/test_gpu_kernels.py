@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from block_sparse_spatiotemporal_b200 import fvattn as F
-from block_sparse_spatiotemporal_b200.inputs import Workload, WORKLOADS, make_inputs
+from block_sparse_spatiotemporal_b200.inputs import f32_to_bf16_bits, Workload, WORKLOADS, make_inputs
 from oracle import fvattn_oracle as O
 from tests.gpu_util import (assert_close, compare_blocks, sum_checks, oracle_coarse, oracle_rope, rope_of, shape_of,
                             to_dev, to_host)
@@ -142,12 +142,42 @@ def _fine_case(wl, layout, top_p=None, k_min=None):
     dict(grid=(8, 16, 16), dtype="bf16", d=128, top_p=0.0, k_min=5),               # fixed top-k
     dict(grid=(8, 8, 12), dtype="bf16", d=128, order="hilbert", rope=True, top_p=0.9, k_min=3),
     dict(grid=(8, 8, 12), dtype="f32", d=128, order="hilbert", rope=True, top_p=0.9, k_min=3),
+    dict(grid=(4, 4, 20), dtype="bf16", d=128, top_p=0.9, k_min=2),                # nT = 5: a one-tile quad
+    dict(grid=(4, 8, 12), dtype="bf16", d=128, top_p=0.5, k_min=1),                # nT = 6: a two-tile quad
+    dict(grid=(4, 4, 28), dtype="bf16", d=128, top_p=0.7, k_min=1),                # nT = 7: a three-tile quad
 ])
 @pytest.mark.parametrize("layout", [F.NATURAL, F.TILED])
 def test_block_sparse_fwd_matches_oracle(case, layout):
     wl = small(case["grid"], d=case["d"], dtype=case["dtype"], order=case.get("order", "raster"),
                rope=case.get("rope", False), gen=case.get("gen", "per_head"))
     _fine_case(wl, layout, case["top_p"], case["k_min"])
+
+
+def test_late_large_logits_rescale():
+    """Keys of the last tile scaled by 2^4 (exact in bf16): with dense lists
+    every row meets logits far above its first tile's only at the last step,
+    so the running max moves up there (O, l and the step's P rescaled)."""
+    wl = small((4, 8, 16), heads=2)                 # nT = 8
+    q, k, v = make_inputs(wl)
+    k = k.copy()
+    pos = O.positions(wl.grid, wl.order)
+    last = pos // 64 == wl.num_tiles - 1
+    big = O.as_f64(k[:, :, last], "bf16") * 16.0
+    k[:, :, last] = f32_to_bf16_bits(big.astype(np.float32))
+    shape = shape_of(wl)
+    ws = F.workspace(shape)
+    nT = wl.num_tiles
+    counts = torch.full((1, wl.heads, nT), nT, dtype=torch.int32, device="cuda")
+    idx = torch.arange(nT, dtype=torch.int32, device="cuda").repeat(1, wl.heads, nT, 1)
+    out, lse = F.block_sparse_fwd(shape, to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), counts, idx, ws)
+    assert F.device_status(ws) == 0
+    full = (np.full(nT, nT), np.tile(np.arange(nT), (nT, 1)))
+    for h in range(wl.heads):
+        r = O.forward_head(q[0, h], k[0, h], v[0, h], wl.grid, wl.order, 1.0, 1, "bf16", blocks=full)
+        s = O.default_scale(wl.head_dim) * np.abs(O.as_f64(q[0, h], "bf16") @ O.as_f64(k[0, h], "bf16").T)
+        assert s.max() * 1.4427 > 64          # the jump exceeds the kernel's headroom somewhere
+        assert_close(to_host(out)[0, h], r["out"], "bf16", f"out head {h}")
+        assert_close(to_host(lse)[0, h], r["lse"], "bf16", f"lse head {h}")
 
 
 def test_single_tile_grid():

@@ -295,9 +295,40 @@ def test_rope_bf16_operand_rounding_only_in_fine_stage():
     qr = O.rope_3d(O.as_f64(q, "bf16"), coords)
     kr = O.rope_3d(O.as_f64(k, "bf16"), coords)
     assert np.abs(res["qp"] - O.pool_tiles(O.to_tiled(qr, res["pos"]))).max() == 0
-    out, lse = O.dense_attention_loop(O.round_bf16(qr).tolist(), O.round_bf16(kr).tolist(),
+    qr32 = O.rope_3d_f32(O.as_f64(q, "bf16"), coords).astype(np.float64)
+    kr32 = O.rope_3d_f32(O.as_f64(k, "bf16"), coords).astype(np.float64)
+    out, lse = O.dense_attention_loop(O.round_bf16(qr32).tolist(), O.round_bf16(kr32).tolist(),
                                       O.as_f64(v, "bf16").tolist(), 1 / math.sqrt(128))
     assert np.abs(res["out"] - np.array(out)).max() < 1e-12
+
+
+def test_rope_f32_rotation_is_the_float32_evaluation_of_the_rotation():
+    """rope_3d_f32 (the fine stage's operand rotation) against the float64
+    rotation: identical at position 0 (cos 1, sin 0 exactly), within two
+    float32 rounding errors of the float64 value elsewhere, pair norms kept
+    to float32 precision, and equal to a scalar loop that rounds every
+    intermediate through struct's IEEE single format."""
+    import struct
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((6, 128)).astype(np.float32).astype(np.float64)
+    coords = np.array([[0, 0, 0], [1, 2, 3], [19, 47, 79], [5, 0, 9], [0, 11, 0], [7, 7, 7]])
+    y = O.rope_3d_f32(x, coords)
+    assert y.dtype == np.float32
+    assert np.array_equal(y[0], x[0].astype(np.float32))
+    ref = O.rope_3d(x, coords)
+    mag = np.abs(x[:, 0::2]) + np.abs(x[:, 1::2])
+    err = np.maximum(np.abs(y[:, 0::2] - ref[:, 0::2]), np.abs(y[:, 1::2] - ref[:, 1::2]))
+    assert (err <= 2 * 2.0 ** -23 * mag + 1e-30).all()
+    n0, n1 = x[:, 0::2] ** 2 + x[:, 1::2] ** 2, y[:, 0::2].astype(np.float64) ** 2 + y[:, 1::2].astype(np.float64) ** 2
+    assert np.abs(n1 - n0).max() <= 1e-5 * n0.max()
+    f = lambda v: struct.unpack("f", struct.pack("f", v))[0]   # noqa: E731
+    r, dim = 2, 50                                             # token 2, h-axis pair j = 3
+    da, j = 42, 3
+    ang = coords[r, 1] * 10000.0 ** (-2.0 * j / da)
+    c, s = f(math.cos(ang)), f(math.sin(ang))
+    x0, x1 = f(x[r, dim]), f(x[r, dim + 1])
+    assert y[r, dim] == f(f(x0 * c) - f(x1 * s))
+    assert y[r, dim + 1] == f(f(x0 * s) + f(x1 * c))
 
 
 def test_rope_each_axis_group_matches_library_1d_rotary():
