@@ -208,12 +208,48 @@ def workload_config(wl, args, world: int = 1) -> dict:
             "parallelism": f"replica x{world}"}
 
 
+def oracle_tiny_single_core() -> dict:
+    """The oracle's whole path (coarse stage and fine stage of every head)
+    on the tiny fp32 workload (8x16x16 tokens, 2 heads, d=64) on one core."""
+    from oracle import fvattn_oracle as O
+    wl1 = WORKLOADS["tiny_fp32"]
+    q, k, v = make_inputs(wl1)
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except Exception:
+        limit = None
+    t0 = time.perf_counter()
+    for h in range(wl1.heads):
+        O.forward_head(q[0, h], k[0, h], v[0, h], wl1.grid, wl1.order, wl1.top_p, wl1.k_min, wl1.dtype)
+    ms = (time.perf_counter() - t0) * 1e3
+    if limit is not None:
+        limit.unregister()
+    return {"workload": wl1.name, "ms": ms, "cores": 1}
+
+
 def cpu_baseline_of(res: dict) -> dict:
     return {"value": res["flops"] / res["est_s"] / 1e12, "unit": UNIT, "cores": res["threads"],
             "nproc": os.cpu_count(), "kind": "oracle", "sample": res["desc"],
             "est_ms_per_step": res["est_s"] * 1e3,
             "stage_ms": {k: v * 1e3 for k, v in res["stage_s"].items()},
             "ms_is": "estimate: the sample's time scaled to the whole workload"}
+
+
+def sm_imbalance(F, shape, ws, rope=None) -> dict:
+    """Load balance of the last profiled fine-stage launch on `ws`: busy time
+    (set-up done to last item finished) of every persistent CTA; the ratio
+    max / mean is the single-GPU counterpart of the per-rank imbalance ratio
+    the load balancing targets."""
+    t = F.profile_cta_times(shape, ws, rope)
+    if len(t) == 0:
+        return None
+    busy = (t[:, 1] - t[:, 0]).astype(np.float64)
+    span = float(t[:, 1].max() - t[:, 0].min())
+    return {"ctas": int(len(t)), "max_over_mean": float(busy.max() / busy.mean()),
+            "mean_busy_us": float(busy.mean() / 1e3), "max_busy_us": float(busy.max() / 1e3),
+            "min_busy_us": float(busy.min() / 1e3), "launch_span_us": span / 1e3,
+            "what": "per-CTA busy time of the persistent fine stage in the last timed step (globaltimer)"}
 
 
 def run_reference(args, wl):
@@ -323,6 +359,7 @@ def run_gpu(args, wl):
     torch.cuda.synchronize(dev)
     F.profile_enable(False)
     stages = F.profile_read()
+    imbalance = None if args.subblock else sm_imbalance(F, shape, ws, rope)
     clocks = sampler.stop() if sampler else None
     if world > 1:
         dist.barrier()
@@ -418,6 +455,7 @@ def run_gpu(args, wl):
                          "frac_sustained": achieved / pk["bf16_tflops_sustained"]
                          if pk.get("bf16_tflops_sustained") else None},
             "gpu_launches": sum(n for _, n in stages.values()),
+            "sm_imbalance": imbalance,
             "clocks": clocks,
             "e2e": e2e,
         }
@@ -426,6 +464,7 @@ def run_gpu(args, wl):
             lists = None if args.subblock else (counts.cpu().numpy(), idx.cpu().numpy())
             res = oracle_sample(wl, q, k, v, budget_s=args.cpu_budget, gpu_lists=lists)
             line["cpu_baseline"] = cpu_baseline_of(res)
+            line["cpu_baseline"]["tiny_single_core"] = oracle_tiny_single_core()
             if res["parity"] is not None:
                 line["parity"] = dict(res["parity"], what="block lists of the timed forward vs the oracle, every "
                                       "row of every head; borderline / near-tie rows that differ must be valid "
@@ -438,8 +477,12 @@ def run_gpu(args, wl):
 
 
 def run_sweep(args):
-    """The 480p sweep: ms, effective TFLOP/s and density at each (top_p, k_min) point, then the
-    cached-mask steps (lists of step 0 reused on perturbed inputs).  One JSON line."""
+    """The 480p sweep (seed 4): at every (top_p, k_min) point -- top-p 0.5 ..
+    1.0 with k_min 8 and fixed top-k 8 / 32 / 128 -- the forward's ms,
+    effective TFLOP/s and density, the informational error of its output
+    against the dense output (top_p = 1) of the same inputs, and cached-mask
+    mode: the point's step-0 lists reused on the ten perturbed steps
+    (Q, K += 0.05 N(0,1) per step, V fixed), each step timed.  One JSON line."""
     import torch
     from block_sparse_spatiotemporal_b200 import fvattn as F
     from block_sparse_spatiotemporal_b200.inputs import perturb_steps, sweep_points
@@ -449,60 +492,58 @@ def run_sweep(args):
     q, k, v, masters = make_inputs(wl, keep_f32_masters=True)
     as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
+    perturbed = [(as_dev(qt), as_dev(kt)) for qt, kt in perturb_steps(wl, masters)]
     shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16)
     ws = F.workspace(shape, device=dev)
     cache, counts, _ = F.new_cache(shape, device=dev)
     out = torch.empty_like(qd)
     lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    points = []
-    for top_p, k_min in sweep_points():
-        def step():
-            F.forward(shape, qd, kd, vd, ws, top_p, k_min, cache=cache, out=out, lse=lse)
+    F.forward(shape, qd, kd, vd, ws, 1.0, 1, cache=cache, out=out, lse=lse)
+    dense = out.float().clone()
+    fl = pair_flops(wl.head_dim)
+    total = wl.heads * wl.num_tiles ** 2
+
+    def timed(fn, n):
         for _ in range(args.warmup):
-            step()
+            fn()
         torch.cuda.synchronize(dev)
-        pairs = int(counts.sum().item())
         F.profile_read()
         F.profile_enable(True)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            step()
+        for _ in range(n):
+            fn()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         F.profile_enable(False)
-        stages = F.profile_read()
+        st = F.profile_read()
         if F.device_status(ws) != 0:
             raise RuntimeError("device status set in the sweep")
-        ms = e0.elapsed_time(e1) / args.steps
-        fine = stages["fine"][0] / max(stages["fine"][1], 1)
-        flops = pairs * pair_flops(wl.head_dim)
+        return e0.elapsed_time(e1) / n, st["fine"][0] / max(st["fine"][1], 1)
+
+    points = []
+    for top_p, k_min in sweep_points():
+        ms, fine = timed(lambda: F.forward(shape, qd, kd, vd, ws, top_p, k_min, cache=cache, out=out, lse=lse),
+                         args.steps)
+        pairs = int(counts.sum().item())      # the cache holds this point's step-0 lists
+        err = (out.float() - dense).abs()
+        cached_ms = []
+        for qx, kx in perturbed:
+            cms, _ = timed(lambda: F.forward(shape, qx, kx, vd, ws, top_p, k_min, cache=cache, reuse_mask=True,
+                                             out=out, lse=lse), max(3, args.steps // 4))
+            cached_ms.append(cms)
         points.append({"top_p": top_p, "k_min": k_min, "ms": ms, "fine_ms": fine,
-                       "tflops": flops / (ms / 1e3) / 1e12, "fine_tflops": flops / (fine / 1e3) / 1e12,
-                       "density": pairs / (wl.heads * wl.num_tiles ** 2)})
-    # cached-mask steps: fill the cache on step 0, then reuse it on the perturbed inputs
-    F.forward(shape, qd, kd, vd, ws, wl.top_p, wl.k_min, cache=cache, out=out, lse=lse)
-    torch.cuda.synchronize(dev)
-    pairs = int(counts.sum().item())
-    cached = []
-    for qt, kt in perturb_steps(wl, masters):
-        qx, kx = as_dev(qt), as_dev(kt)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            F.forward(shape, qx, kx, vd, ws, wl.top_p, wl.k_min, cache=cache, reuse_mask=True, out=out, lse=lse)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        cached.append(e0.elapsed_time(e1) / args.steps)
-    if F.device_status(ws) != 0:
-        raise RuntimeError("device status set in the cached steps")
+                       "tflops": pairs * fl / (ms / 1e3) / 1e12, "fine_tflops": pairs * fl / (fine / 1e3) / 1e12,
+                       "density": pairs / total, "selected_pairs": pairs,
+                       "err_vs_dense": {"max_abs": float(err.max().item()), "mean_abs": float(err.mean().item())},
+                       "cached_mask": {"steps": len(cached_ms), "ms_per_step": cached_ms,
+                                       "ms_mean": statistics.mean(cached_ms),
+                                       "tflops_mean": pairs * fl / (statistics.mean(cached_ms) / 1e3) / 1e12}})
     line = {"metric": METRIC, "unit": UNIT, "workload": wl.name, "steps": args.steps, "warmup": args.warmup,
-            "sweep": points,
-            "cached_mask": {"top_p": wl.top_p, "k_min": wl.k_min,
-                            "density": pairs / (wl.heads * wl.num_tiles ** 2), "ms_per_step": cached,
-                            "tflops_mean": pairs * pair_flops(wl.head_dim) / (statistics.mean(cached) / 1e3) / 1e12}}
+            "dtype": "bf16", "data": "synthetic",
+            "dense_reference": "the forward at top_p = 1 (every key tile) on the same step-0 inputs",
+            "sweep": points}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -807,7 +848,8 @@ def run_augment(args, wl):
             raise RuntimeError("device status set")
         res[name] = {"ms": e0.elapsed_time(e1) / args.steps,
                      "fine_ms": st["fine"][0] / max(st["fine"][1], 1),
-                     "stage_ms": {k2: round(v2[0] / args.steps, 4) for k2, v2 in st.items() if v2[1]}}
+                     "stage_ms": {k2: round(v2[0] / args.steps, 4) for k2, v2 in st.items() if v2[1]},
+                     "sm_imbalance": sm_imbalance(F, shape, ws, rope)}
     pairs = int(base[0].sum().item())
     apairs = int(aug[0].sum().item())
     fl = pair_flops(wl.head_dim)

@@ -108,6 +108,7 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   L.rank = take(sizeof(int) * (size_t)g.BH * g.P);
   L.useg = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.qcost = take(sizeof(int) * (size_t)g.BH * g.Qn);
+  L.cta_times = take(sizeof(unsigned long long) * (1 + 2 * (size_t)kMaxCtas));
   const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
   L.qrot = take(rot);
   L.krot = take(rot);
@@ -299,6 +300,12 @@ Profiler& prof() {
   return p;
 }
 
+bool profiling() {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lock(p.mu);
+  return p.on;
+}
+
 // Records events around one launch when profiling is on.
 struct StageTimer {
   int stage;
@@ -467,6 +474,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     FV_TRY(make_tile_map(&mv, v, c.g, natural));
     FineQArgs a{};
     a.g = c.g;
+    a.cta_times = profiling() ? c.at<unsigned long long>(c.L.cta_times) : nullptr;
     a.uni = c.at<int>(c.L.uni);
     a.ucount = c.at<int>(c.L.ucount);
     a.useg = c.at<int>(c.L.useg);
@@ -493,6 +501,7 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     FV_TRY(make_tile_map(&mv, v, c.g, natural));
     FineTcArgs a{};
     a.g = c.g;
+    a.cta_times = profiling() ? c.at<unsigned long long>(c.L.cta_times) : nullptr;
     a.uni = c.at<int>(c.L.uni);
     a.ucount = c.at<int>(c.L.ucount);
     a.worklist = worklist ? worklist : c.at<int>(c.L.worklist);
@@ -966,6 +975,26 @@ int fvattn_profile_read(double* ms, int64_t* launches) {
     if (launches) launches[i] = cnt[i];
   }
   return st;
+}
+
+int fvattn_profile_cta_times(const fvattn_shape* shape, const fvattn_rope* rope, void* ws, fvattn_stream_t stream,
+                             int64_t* ns, int32_t capacity, int32_t* num_ctas) {
+  if (!ws || !ns || !num_ctas || capacity < 0) return FVATTN_ERR_INVALID_ARG;
+  Geom g{};
+  FV_TRY(make_geom(shape, &g));
+  FV_TRY(check_rope(rope, g));
+  const WsLayout L = layout_for(g, shape->dtype, rope);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FV_CUDA(cudaStreamSynchronize(s));
+  unsigned long long n = 0;
+  const char* base = static_cast<const char*>(ws) + L.cta_times;
+  FV_CUDA(cudaMemcpy(&n, base, sizeof(n), cudaMemcpyDeviceToHost));
+  if (n > (unsigned long long)kMaxCtas) return FVATTN_ERR_DEVICE;
+  const int32_t m = (int32_t)n < capacity ? (int32_t)n : capacity;
+  if (m > 0) FV_CUDA(cudaMemcpy(ns, base + sizeof(unsigned long long), sizeof(int64_t) * 2 * (size_t)m,
+                                cudaMemcpyDeviceToHost));
+  *num_ctas = (int32_t)n;
+  return FVATTN_OK;
 }
 
 const char* fvattn_status_string(int status) {

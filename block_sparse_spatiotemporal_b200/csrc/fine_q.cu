@@ -21,9 +21,10 @@
 //                in TMEM as soon as PV_h(c-1) has been issued, and the
 //                softmax of one half runs while the tensor core works on
 //                the other half's products (ping-pong);
-//   warps 4-7    softmax and epilogue of half A, warps 8-11 of half B:
-//                thread r owns row r of its half (TMEM lane r) and all 128
-//                keys of a step.
+//   warps 2-5    softmax and epilogue of half A, warps 6-9 of half B:
+//                thread r owns row r of its half (TMEM lane r, the lane
+//                quarter of warp w being w mod 4) and all 128 keys of a
+//                step, loaded from TMEM at once.
 // Online softmax in base 2 with a lazy rescale: a row keeps its reference
 // max m (set by its first selected key tile) until a key tile's largest
 // logit exceeds it by more than 64 (in log2 units); then m moves up by a
@@ -46,8 +47,8 @@ namespace fq {
 constexpr int D = 128;
 constexpr int KST = 3;                                  // K ring depth
 constexpr int VST = 2;                                  // V ring depth
-constexpr int THREADS = 384;
-constexpr int SM_WARP0 = 4;                             // first softmax warp
+constexpr int THREADS = 320;
+constexpr int SM_WARP0 = 2;                             // first softmax warp
 constexpr uint32_t BOX = 64 * 128;                      // one 64-row x 128-byte box: 8 KB
 constexpr uint32_t QH_BYTES = 4 * BOX;                  // one half: 2 tiles x 2 d-halves: 32 KB
 constexpr uint32_t QH_DHALF = 2 * BOX;                  // one d-half of a half's 128 rows
@@ -187,6 +188,111 @@ __device__ inline float fq_exp64(const uint32_t (&s0)[32], const uint32_t (&s1)[
   return (a0 + a1) + (a2 + a3);
 }
 
+// tcgen05.wait::ld that also names the destination registers of the loads it
+// waits for, so the compiler cannot move their first use above the wait.
+__device__ inline void fq_wait_ld(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]),
+        "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+        "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ inline void fq_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ inline void fq_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Largest logit of 32 keys.
+__device__ inline float fq_max32(const uint32_t (&s)[32]) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    m0 = fq_max3(m0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+    m1 = fq_max3(m1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+  }
+  return fmaxf(m0, m1);
+}
+
+// Pairs of a 32-key chunk (16 pairs) whose exponentials run on the FMA
+// pipe (exp2 by a polynomial) instead of the MUFU unit: 0, every 4th, or
+// every 2nd pair.
+#ifndef FVATTN_FQ_POLY
+#define FVATTN_FQ_POLY 0
+#endif
+__host__ __device__ constexpr bool fq_poly_pair(int i) {
+  return FVATTN_FQ_POLY == 4 ? (i & 3) == 3 : FVATTN_FQ_POLY == 2 ? (i & 1) == 1 : false;
+}
+
+// 2^x for a pair on the FMA pipe: x clamped to [-126, 126]; i = floor(x)
+// from a round-down add of 1.5 * 2^23 (the low mantissa bits of the sum
+// hold i), f = x - i in [0, 1), 2^f by a degree-3 polynomial, i added to the
+// exponent field.  The coefficients are a minimax fit of 2^f on [0, 1) in
+// relative error (a linear program over a dense grid): max relative error
+// 7.5e-5, below half a bf16 ulp (2^-9), the precision P is stored in.
+__device__ inline void fq_exp2_poly(float x0, float x1, float& y0, float& y1) {
+  constexpr float C0 = 0.9999252557754517f, C1 = 0.6958333253860474f, C2 = 0.22606715559959412f,
+                  C3 = 0.07802474498748779f, MAGIC = 12582912.f;
+  x0 = fminf(fmaxf(x0, -126.f), 126.f);
+  x1 = fminf(fmaxf(x1, -126.f), 126.f);
+  uint64_t X = fq_f2(x0, x1), M = fq_f2(MAGIC, MAGIC), Y, F;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(Y) : "l"(X), "l"(M));
+  uint64_t YM;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(YM) : "l"(Y), "l"(M));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(F) : "l"(X), "l"(YM));
+  uint64_t P = fq_fma2(F, fq_f2(C3, C3), fq_f2(C2, C2));
+  P = fq_fma2(P, F, fq_f2(C1, C1));
+  P = fq_fma2(P, F, fq_f2(C0, C0));
+  float p0, p1, q0, q1;
+  fq_uf2(P, p0, p1);
+  fq_uf2(Y, q0, q1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(q0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(q1) << 23));
+}
+
+// P = 2^(s * sl2 - m) of 32 keys as 16 bf16x2 words; returns their sum.
+__device__ inline float fq_exp32(const uint32_t (&s)[32], float sl2, float m, uint32_t (&pk)[16]) {
+  const uint64_t SL = fq_f2(sl2, sl2), NM = fq_f2(-m, -m);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1, p0, p1;
+    fq_uf2(fq_fma2(fq_f2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), SL, NM), x0, x1);
+    if (fq_poly_pair(i)) {
+      fq_exp2_poly(x0, x1, p0, p1);
+    } else {
+      p0 = fq_ex2(x0);
+      p1 = fq_ex2(x1);
+    }
+    const uint32_t w = fq_bf16x2(p0, p1);
+    pk[i] = w;
+    if (i & 1) {
+      a2 = fq_add_lo(a2, w);
+      a3 = fq_add_hi(a3, w);
+    } else {
+      a0 = fq_add_lo(a0, w);
+      a1 = fq_add_hi(a1, w);
+    }
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
 // 2^k for an integer k in [-126, 127], exact.
 __device__ inline float fq_pow2i(int k) { return __int_as_float((127 + k) << 23); }
 
@@ -268,6 +374,7 @@ __global__ void __launch_bounds__(fq::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = ctl->tmem_base;
+  const unsigned long long t_start = threadIdx.x == 0 && a.cta_times ? global_ns() : 0ull;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
@@ -415,18 +522,15 @@ __global__ void __launch_bounds__(fq::THREADS, 1)
       first_in_item[0] = first_in_item[1] = true;
       for (int i = 0; i < steps; ++i, ++c) {
         const int ks = (int)(c % KST);
-        // PV_A of the previous step needs only its V and P_A
-        if (prev_act && !mbar_wait_warp(&ctl->v_full[prev_vs], (uint32_t)(prev_c / VST) & 1, abort_flag, a.status,
-                                        cap)) {
+        // K(c) (and the item's Q) and V(c-1) first, so that PV_A(c-1) and S_A(c) go out back to back
+        if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(c / KST) & 1, abort_flag, a.status, cap) ||
+            (i == 0 && !mbar_wait_warp(&ctl->q_full, (uint32_t)kq & 1, abort_flag, a.status, cap)) ||
+            (prev_act && !mbar_wait_warp(&ctl->v_full[prev_vs], (uint32_t)(prev_c / VST) & 1, abort_flag,
+                                         a.status, cap))) {
           ok = false;
           break;
         }
         if ((prev_act & 1) && !issue_pv(0)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(c / KST) & 1, abort_flag, a.status, cap) ||
-            (i == 0 && !mbar_wait_warp(&ctl->q_full, (uint32_t)kq & 1, abort_flag, a.status, cap))) {
           ok = false;
           break;
         }
@@ -516,44 +620,54 @@ __global__ void __launch_bounds__(fq::THREADS, 1)
         }
         tc_fence_after();
         const int info = ctl->info[h];
-#pragma unroll 1
-        for (int t = 0; t < 2; ++t) {
-          const bool sel = (info >> (4 * t + qsel)) & 1;
-          uint32_t pk[32];
+        // four chunks of 32 keys (chunks 2t, 2t+1 = key tile t), all loaded at once; P of chunk j
+        // (16 bf16x2 words) goes to columns 16 j .. 16 j + 15, over S values already read
+        // chunks 0-2 are loaded at once; chunk 3 goes into chunk 0's registers once chunk 0 is done
+        // and lands while chunks 1 and 2 are computed
+        uint32_t sc[3][32];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) tmem_ld32(tS + 32 * j, sc[j]);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) fq_wait_ld(sc[j]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j == 1) tmem_ld32(tS + 96, sc[0]);
+          if (j == 3) fq_wait_ld(sc[0]);
+          const bool sel = (info >> (4 * (j >> 1) + qsel)) & 1;
+          uint32_t pk[16];
           float alpha = 1.f;
           bool rescale = false;
-          {
-            uint32_t s0[32], s1[32];
-            tmem_ld32(tS + 64 * t, s0);
-            tmem_ld32(tS + 64 * t + 32, s1);
-            tmem_wait_ld();
-            if (sel) {
-              const float mx = fq_max64(s0, s1) * sl2;
-              if (m_use == -INFINITY) {
-                m_use = mx;                     // first selected key tile of the row
-              } else if (mx > m_use + RESCALE_X) {
-                // move the reference max up by a whole power of two
-                const int k = (int)ceilf(mx - m_use);
-                alpha = fq_pow2i(-(k < 126 ? k : 126));
-                m_use += (float)k;
-                rescale = true;
-              }
-              l = l * alpha + fq_exp64(s0, s1, sl2, m_use, pk);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) pk[i] = 0u;
+          if (sel) {
+            const float mx = fq_max32(sc[j == 3 ? 0 : j]) * sl2;
+            if (m_use == -INFINITY) {
+              m_use = mx;                       // first selected chunk of the row
+            } else if (mx > m_use + RESCALE_X) {
+              // move the reference max up by a whole power of two
+              const int k = (int)ceilf(mx - m_use);
+              alpha = fq_pow2i(-(k < 126 ? k : 126));
+              m_use += (float)k;
+              rescale = true;
             }
+            l = l * alpha + fq_exp32(sc[j == 3 ? 0 : j], sl2, m_use, pk);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
           }
           if (__any_sync(0xffffffffu, rescale)) {
-            // P of key tile 0 of this step is already in TMEM (t == 1), and O holds the PVs of the
-            // earlier steps of this item: scale both by alpha (1 on the rows that keep their max)
-            if (t == 1) {
-              uint32_t p0[32];
-              tmem_wait_st();
-              tmem_ld32(tS, p0);
+            // P of the earlier chunks of this step is in TMEM, and O holds the PVs of the earlier
+            // steps of this item: scale both by alpha (1 on the rows that keep their max)
+            tmem_wait_st();
+#pragma unroll 1
+            for (int jj = 0; jj < j; ++jj) {
+              uint32_t p0[16];
+              fq_ld16(tS + 16 * jj, p0);
               tmem_wait_ld();
-              fq_scale_bf16(p0, alpha);
-              tmem_st32(tS, p0);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float lo = __uint_as_float(p0[i] << 16) * alpha, hi = __uint_as_float(p0[i] & 0xFFFF0000u) * alpha;
+                p0[i] = fq_bf16x2(lo, hi);
+              }
+              fq_st16(tS + 16 * jj, p0);
             }
             if (st > 0) {
               if (!mbar_wait(&ctl->pv_done[h], (uint32_t)(ch - 1) & 1, abort_flag, a.status, cap)) {
@@ -572,8 +686,9 @@ __global__ void __launch_bounds__(fq::THREADS, 1)
               }
             }
           }
-          tmem_st32(tS + 32 * t, pk);
+          fq_st16(tS + 16 * j, pk);
         }
+
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
@@ -614,6 +729,12 @@ __global__ void __launch_bounds__(fq::THREADS, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0 && a.cta_times && blockIdx.x < kMaxCtas) {
+    // busy time of this CTA: setup done to its last item finished
+    a.cta_times[1 + 2 * blockIdx.x] = t_start;
+    a.cta_times[2 + 2 * blockIdx.x] = global_ns();
+    if (blockIdx.x == 0) a.cta_times[0] = gridDim.x;
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, fq::TMEM_COLS);

@@ -348,6 +348,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = ctl->tmem_base;
+  const unsigned long long t_start = threadIdx.x == 0 && a.cta_times ? global_ns() : 0ull;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
@@ -825,6 +826,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0 && a.cta_times && blockIdx.x < kMaxCtas) {
+    // busy time of this CTA: setup done to its last item finished
+    a.cta_times[1 + 2 * blockIdx.x] = t_start;
+    a.cta_times[2 + 2 * blockIdx.x] = global_ns();
+    if (blockIdx.x == 0) a.cta_times[0] = gridDim.x;
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, ft::TMEM_COLS);

@@ -18,6 +18,14 @@ constexpr int kTileTokens = 64;
 constexpr int kItemTiles = 2;   // query tiles per fine-stage work item (one 128-row tile)
 constexpr int kSubBlocks = 8;   // 2x2x2 sub-cubes of a tile in sub-block scoring
 constexpr int kMaxTiles = 8192;
+constexpr int kMaxCtas = 1024;  // persistent grid bound (fine-stage CTA time record)
+
+// Global nanosecond timer (the same clock on every SM).
+__device__ inline unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 // Device status codes (workspace status word).
 constexpr int kStatusBadBlock = 1;
@@ -56,6 +64,7 @@ struct WsLayout {
   size_t uni, ucount;    // int32 [BH*P*nT], [BH*P]
   size_t worklist;       // int32 [BH*P]
   size_t useg, qcost;    // int32 [BH*Qn] quad items: union segments and cost
+  size_t cta_times;      // u64 [1 + 2 * kMaxCtas] fine-stage CTA start / end times (profiling)
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
@@ -91,6 +100,7 @@ struct ScoreArgs {
 
 struct FineTcArgs {
   Geom g;
+  unsigned long long* cta_times;   // optional: [0] = CTAs, then per CTA (start, end) in ns
   const int* uni;
   const int* ucount;
   const int* worklist;
@@ -107,6 +117,7 @@ struct FineTcArgs {
 // Fine stage over quad items (four query tiles in two 128-row halves).
 struct FineQArgs {
   Geom g;
+  unsigned long long* cta_times;   // optional: [0] = CTAs, then per CTA (start, end) in ns
   const int* uni;        // [items][nT] union entries (key tile | selection bits << 16)
   const int* ucount;     // [items] entries
   const int* useg;       // [items] entries of both halves | entries of half A only << 16

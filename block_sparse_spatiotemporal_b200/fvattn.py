@@ -22,7 +22,7 @@ __all__ = [
     "pool_select_subblock",
     "tile_reorder", "pool_select", "build_worklist", "block_sparse_fwd", "forward",
     "device_status", "selftest_wait_timeout", "new_blocks", "new_cache", "profile_enable", "profile_read",
-    "STAGES", "pool_select_noalloc", "noalloc_status", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
+    "STAGES", "pool_select_noalloc", "noalloc_status", "profile_cta_times", "workspace_size_qkv", "qkv_rope", "workspace_size_bwd", "block_sparse_bwd",
     "augment_lists", "block_sparse_fwd_worklist", "timestep_params",
 ]
 
@@ -89,6 +89,8 @@ _SIGS = {
     "fvattn_pool_select_noalloc": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
                                    ctypes.c_float, ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p],
     "fvattn_pool_select_noalloc_status": [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)],
+    "fvattn_profile_cta_times": [ctypes.POINTER(Shape), ctypes.POINTER(Rope), ctypes.c_void_p, ctypes.c_void_p,
+                                 ctypes.POINTER(ctypes.c_int64), ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
     "fvattn_build_worklist": [ctypes.POINTER(Shape), ctypes.POINTER(Blocks), ctypes.c_void_p, ctypes.c_void_p,
                               ctypes.c_size_t, ctypes.c_void_p],
     "fvattn_block_sparse_fwd": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -420,6 +422,19 @@ def selftest_wait_timeout(ws, cap_iterations: int, stream=None):
 def profile_enable(on: bool = True):
     """Record CUDA events around every library kernel (per-stage timing)."""
     _check("fvattn_profile_enable", lib().fvattn_profile_enable(1 if on else 0))
+
+
+def profile_cta_times(shape: Shape, ws, rope: Optional[Rope] = None, stream=None):
+    """(start, end) nanoseconds of every CTA of the last profiled fine-stage
+    launch that used `ws`, as an [n, 2] int64 numpy array (synchronises)."""
+    import numpy as np
+    cap = 1024
+    buf = (ctypes.c_int64 * (2 * cap))()
+    n = ctypes.c_int32(0)
+    _check("fvattn_profile_cta_times", lib().fvattn_profile_cta_times(ctypes.byref(shape), _rope_ptr(rope), _ptr(ws),
+                                                                        _stream(stream), buf, cap, ctypes.byref(n)))
+    m = min(n.value, cap)
+    return np.frombuffer(buf, dtype=np.int64, count=2 * m).reshape(m, 2).copy()
 
 
 def profile_read():

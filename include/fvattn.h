@@ -344,6 +344,19 @@ typedef enum {
 int fvattn_profile_enable(int enable);
 int fvattn_profile_read(double* ms, int64_t* launches);
 
+/* Per-CTA busy time of the persistent fine stage, the single-GPU analogue of
+ * the per-rank load the "FVAttn" digest balances (section 02; section 03
+ * reports the mean imbalance ratio).  While profiling is enabled, every
+ * fine-stage launch of a call records, for each CTA, the global-timer
+ * nanoseconds when its set-up was done and when its last item finished, in
+ * the call's workspace.  This reads the record of the last such launch that
+ * used workspace `ws` (a DEVICE pointer; shape and rope as in that call, to
+ * locate the record): it synchronises `stream`, writes 2 * min(n, capacity)
+ * int64 (start, end pairs) to the HOST array `ns` and n (the grid size) to
+ * *num_ctas.  Returns FVATTN_ERR_DEVICE if the record is not valid. */
+int fvattn_profile_cta_times(const fvattn_shape* shape, const fvattn_rope* rope, void* ws,
+                             fvattn_stream_t stream, int64_t* ns, int32_t capacity, int32_t* num_ctas);
+
 const char* fvattn_status_string(int status);
 
 #ifdef __cplusplus
