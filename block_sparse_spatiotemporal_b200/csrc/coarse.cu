@@ -61,10 +61,12 @@ __device__ inline void rope_pair(const RopeArgs& r, const Geom& g, int dim, int 
 }
 
 // --------------------------------------------------------------------------
-// Pool: one block per (tile, head, tensor).  4 warps; warp w reads rows
-// w, w+4, ..., each lane DPL consecutive dims of the row (a warp reads one
-// whole row per step).  Sums are fp32 in a fixed order: rows of a warp in
-// sequence, then the 4 warp partials in warp order; mean = sum / 64.
+// Pool: one block per (tile, head, tensor).  4 warps; every lane loads 16
+// bytes (8 bf16 or 4 fp32 dims) of a token row per load, so a warp load
+// covers one or more whole rows; a lane's loads for the whole tile are
+// issued before any of them is summed.  Sums are fp32 in a fixed order:
+// a lane's rows in sequence, then the lanes of a warp that hold the same
+// dims (butterfly), then the 4 warp partials in warp order; mean = sum / 64.
 // The mean is stored as two tf32 values, hi = rn_tf32(mean) and
 // lo = rn_tf32(mean - hi) (the subtraction is exact), row-major [BH][nT][d],
 // the operands of the tensor-core score kernel.  Optionally writes the
@@ -81,7 +83,10 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
                                                    int natural, const int* __restrict__ tile_cube,
                                                    const int* __restrict__ tile_tok, RopeArgs rope, PooledOut po,
                                                    T* __restrict__ qrot, T* __restrict__ krot) {
-  constexpr int DPL = D / 32;
+  constexpr int DPL = 16 / sizeof(T);        // elements per 128-bit load
+  constexpr int LPR = D / DPL;               // lanes per token row
+  constexpr int RPL = 32 / LPR;              // rows per warp load
+  constexpr int ITER = kTileTokens / (4 * RPL);
   __shared__ float part[4][D];
   const int j = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const T* x = which == 0 ? q : k;
@@ -89,33 +94,47 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
   float* lo = po.lo[which];
   T* rot = which == 0 ? qrot : krot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / LPR, col = (lane % LPR) * DPL;
   const int cube = tile_cube[j];
   float acc[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-#pragma unroll 4
-  for (int r = warp; r < kTileTokens; r += 4) {
+  // warp w, iteration it: rows (it * 4 + w) * RPL + sub; all ITER loads of a lane issued before the sums
+  float v[ITER][DPL];
+#pragma unroll
+  for (int it = 0; it < ITER; ++it) {
+    const int r = (it * 4 + warp) * RPL + sub;
     const int n = natural ? cube_row_token(g, cube, r) : j * kTileTokens + r;
-    const T* row = x + ((size_t)bh * g.N + n) * D + lane * DPL;
-    float v[DPL];
-    Vec<T, DPL>::load(row, v);
+    Vec<T, DPL>::load(x + ((size_t)bh * g.N + n) * D + col, v[it]);
+  }
+#pragma unroll
+  for (int it = 0; it < ITER; ++it) {
+    const int r = (it * 4 + warp) * RPL + sub;
     if (rope.enabled) {
       // grid coordinate of the token in this row (tiled rows follow the order)
+      const int n = natural ? cube_row_token(g, cube, r) : j * kTileTokens + r;
       const int nn = natural ? n : tile_tok[j * kTileTokens + r];
       const int t = nn / (g.Hg * g.W), h = (nn / g.W) % g.Hg, w = nn % g.W;
 #pragma unroll
-      for (int i = 0; i < DPL; i += 2) rope_pair(rope, g, lane * DPL + i, t, h, w, v[i], v[i + 1]);
+      for (int i = 0; i < DPL; i += 2) rope_pair(rope, g, col + i, t, h, w, v[it][i], v[it][i + 1]);
     }
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) acc[i] += v[i];
+    for (int i = 0; i < DPL; ++i) acc[i] += v[it][i];
     if (rot) {
-      T* dst = rot + ((size_t)bh * g.N + (size_t)j * kTileTokens + r) * D + lane * DPL;
-      Vec<T, DPL>::store(dst, v);
+      T* dst = rot + ((size_t)bh * g.N + (size_t)j * kTileTokens + r) * D + col;
+      Vec<T, DPL>::store(dst, v[it]);
     }
   }
   if (!hi) return;
+  // lanes holding the same dims (one per row of a warp load) combine in a fixed order
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = acc[i];
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  if (sub == 0) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) part[warp][col + i] = acc[i];
+  }
   __syncthreads();
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
     const float mean = (((part[0][c] + part[1][c]) + part[2][c]) + part[3][c]) * (1.0f / 64.0f);

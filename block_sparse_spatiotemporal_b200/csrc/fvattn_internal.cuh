@@ -228,7 +228,10 @@ template <int DPL> struct Vec<__nv_bfloat16, DPL> {
   static_assert(DPL % 2 == 0, "bf16 rows are read in pairs");
   static __device__ inline void load(const __nv_bfloat16* p, float (&v)[DPL]) {
     uint32_t w[DPL / 2];
-    if constexpr (DPL == 4) {
+    if constexpr (DPL == 8) {
+      const uint4 t = *reinterpret_cast<const uint4*>(p);
+      w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    } else if constexpr (DPL == 4) {
       const uint2 t = *reinterpret_cast<const uint2*>(p);
       w[0] = t.x; w[1] = t.y;
     } else {
@@ -248,7 +251,9 @@ template <int DPL> struct Vec<__nv_bfloat16, DPL> {
       __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t*>(&b);
     }
-    if constexpr (DPL == 4) {
+    if constexpr (DPL == 8) {
+      *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if constexpr (DPL == 4) {
       *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
     } else {
 #pragma unroll
