@@ -168,11 +168,7 @@ __device__ inline float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
-__device__ inline int warp_isum(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
+__device__ inline int warp_isum(int v) { return __reduce_add_sync(0xffffffffu, v); }
 
 // Unsigned key with the order of the float (no NaNs expected).
 __device__ inline uint32_t order_key(float v) {
@@ -244,14 +240,11 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
         bj = i * 32 + lane;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-      if (ov > bv || (ov == bv && oj < bj)) {
-        bv = ov;
-        bj = oj;
-      }
+    // warp argmax in two single-instruction reductions: the largest key, then
+    // the lowest id holding it (a lane's own ties already went to its lowest id)
+    {
+      const uint32_t kmx = __reduce_max_sync(0xffffffffu, order_key(bv));
+      bj = (int)__reduce_min_sync(0xffffffffu, order_key(bv) == kmx ? (uint32_t)bj : 0x7fffffffu);
     }
     if (bj == 0x7fffffff) break;
     if ((bj & 31) == lane) {

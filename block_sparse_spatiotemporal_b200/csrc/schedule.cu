@@ -167,14 +167,20 @@ __global__ void __launch_bounds__(128) quad_union_kernel(Geom g, int Qn, const i
 }
 
 // Longest-first work list by a counting sort on the cost: bins of equal
-// cost in descending order, items inside a bin in ascending code (head-major,
-// so the CTAs that start together share a head's K/V in L2).  One block:
-// histogram, a descending exclusive scan by one warp, then one warp places
-// the items 32 at a time in code order (ranks among equal costs from
-// __match_any_sync), which keeps the order stable and deterministic.
-__global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ cost, int n, int maxc,
-                                                        int* __restrict__ worklist) {
+// cost in descending order, items inside a bin in ascending code.  Items
+// are taken in groups of consecutive codes (one block per group; a group of
+// whole heads keeps the CTAs that run together on a few heads' K/V, which
+// then stay in L2): histogram, a descending exclusive scan by one warp,
+// then one warp places the group's items 32 at a time in code order (ranks
+// among equal costs from __match_any_sync), stable and deterministic.
+__global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ cost_all, int n_all, int group, int maxc,
+                                                        int* __restrict__ worklist_all) {
   extern __shared__ int hist[];  // maxc + 1 bins
+  // block b orders the items [b * group, min(n_all, (b + 1) * group)) among themselves
+  const int first = blockIdx.x * group;
+  const int n = min(group, n_all - first);
+  const int* cost = cost_all + first;
+  int* worklist = worklist_all + first;
   const int tid = threadIdx.x, lane = tid & 31;
   for (int i = tid; i <= maxc; i += blockDim.x) hist[i] = 0;
   __syncthreads();
@@ -204,7 +210,7 @@ __global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ 
     const int base = valid ? hist[c] : 0;
     __syncwarp();
     if (valid) {
-      worklist[base + rank] = i;
+      worklist[base + rank] = first + i;
       if ((peers >> lane) == 1u) hist[c] = base + __popc(peers);   // the group's highest lane advances the bin
     }
     __syncwarp();
@@ -219,7 +225,7 @@ cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const
   quad_union_kernel<<<(unsigned)((items + 3) / 4), 128, (size_t)4 * 4 * words * sizeof(uint32_t), s>>>(
       g, Qn, counts, idx, cap, uni, ucount, useg, qcost, status);
   const int maxc = 2 * ((g.nT + 1) / 2) + 2;
-  lpt_sort_kernel<<<1, 1024, (size_t)(maxc + 1) * sizeof(int), s>>>(qcost, (int)items, maxc, worklist);
+  lpt_sort_kernel<<<1, 1024, (size_t)(maxc + 1) * sizeof(int), s>>>(qcost, (int)items, (int)items, maxc, worklist);
   return cudaGetLastError();
 }
 
@@ -232,9 +238,11 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
   return cudaGetLastError();
 }
 
-cudaError_t launch_rank(const int* key, int n, int max_key, int* worklist, cudaStream_t s) {
+cudaError_t launch_rank(const int* key, int n, int max_key, int group, int* worklist, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  lpt_sort_kernel<<<1, 1024, (size_t)(max_key + 1) * sizeof(int), s>>>(key, n, max_key, worklist);
+  if (group <= 0 || group > n) group = n;
+  lpt_sort_kernel<<<(n + group - 1) / group, 1024, (size_t)(max_key + 1) * sizeof(int), s>>>(key, n, group, max_key,
+                                                                                          worklist);
   return cudaGetLastError();
 }
 
