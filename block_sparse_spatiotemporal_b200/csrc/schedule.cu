@@ -170,51 +170,97 @@ __global__ void __launch_bounds__(128) quad_union_kernel(Geom g, int Qn, const i
 // cost in descending order, items inside a bin in ascending code.  Items
 // are taken in groups of consecutive codes (one block per group; a group of
 // whole heads keeps the CTAs that run together on a few heads' K/V, which
-// then stay in L2): histogram, a descending exclusive scan by one warp,
-// then one warp places the group's items 32 at a time in code order (ranks
-// among equal costs from __match_any_sync), stable and deterministic.
+// then stay in L2).  A block splits its group into `segs` consecutive
+// segments, one warp each: per-segment histograms, per-bin offsets of every
+// segment (bins in descending cost, segments in order), then each warp
+// places its segment's items 32 at a time in code order (ranks among equal
+// costs from __match_any_sync): stable and deterministic.
 __global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ cost_all, int n_all, int group, int maxc,
-                                                        int* __restrict__ worklist_all) {
-  extern __shared__ int hist[];  // maxc + 1 bins
-  // block b orders the items [b * group, min(n_all, (b + 1) * group)) among themselves
+                                                        int segs, int* __restrict__ worklist_all) {
+  extern __shared__ int sort_smem[];
+  int* hist = sort_smem;                         // [segs][maxc + 1]: counts, then running offsets
+  int* base = sort_smem + segs * (maxc + 1);     // [maxc + 1]: items of larger cost
   const int first = blockIdx.x * group;
   const int n = min(group, n_all - first);
   const int* cost = cost_all + first;
   int* worklist = worklist_all + first;
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int i = tid; i <= maxc; i += blockDim.x) hist[i] = 0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bins = maxc + 1;
+  const int seg = (n + segs - 1) / segs;
+  for (int i = tid; i < segs * bins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int i = tid; i < n; i += blockDim.x) atomicAdd(&hist[min(max(cost[i], 0), maxc)], 1);
+  if (warp < segs) {
+    const int lo = warp * seg, hi = min(n, lo + seg);
+    for (int i = lo + lane; i < hi; i += 32) atomicAdd(&hist[warp * bins + min(max(cost[i], 0), maxc)], 1);
+  }
   __syncthreads();
-  if (tid >= 32) return;
-  int run = 0;
-  for (int c0 = maxc; c0 >= 0; c0 -= 32) {
-    const int c = c0 - lane;
-    const int v = c >= 0 ? hist[c] : 0;
-    int x = v;
+  for (int c = tid; c < bins; c += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < segs; ++w) t += hist[w * bins + c];
+    base[c] = t;
+  }
+  __syncthreads();
+  if (warp == 0) {   // descending exclusive scan of the bin totals
+    int run = 0;
+    for (int c0 = maxc; c0 >= 0; c0 -= 32) {
+      const int c = c0 - lane;
+      const int v = c >= 0 ? base[c] : 0;
+      int x = v;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (c >= 0) base[c] = run + x - v;
+      run += __shfl_sync(0xffffffffu, x, 31);
     }
-    if (c >= 0) hist[c] = run + x - v;
-    run += __shfl_sync(0xffffffffu, x, 31);
   }
-  __syncwarp();
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
-    const bool valid = i < n;
-    const int c = valid ? min(max(cost[i], 0), maxc) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, c);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int base = valid ? hist[c] : 0;
-    __syncwarp();
-    if (valid) {
-      worklist[base + rank] = first + i;
-      if ((peers >> lane) == 1u) hist[c] = base + __popc(peers);   // the group's highest lane advances the bin
+  __syncthreads();
+  for (int c = tid; c < bins; c += blockDim.x) {   // each segment's first position in each bin
+    int off = base[c];
+    for (int w = 0; w < segs; ++w) {
+      const int h = hist[w * bins + c];
+      hist[w * bins + c] = off;
+      off += h;
     }
-    __syncwarp();
   }
+  __syncthreads();
+  if (warp < segs) {
+    int* offs = hist + warp * bins;
+    const int lo = warp * seg, hi = min(n, lo + seg);
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < hi;
+      const int c = valid ? min(max(cost[i], 0), maxc) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int pos0 = valid ? offs[c] : 0;
+      __syncwarp();
+      if (valid) {
+        worklist[pos0 + rank] = first + i;
+        if ((peers >> lane) == 1u) offs[c] = pos0 + __popc(peers);   // the group's highest lane advances the bin
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Segments per block such that the histograms fit in 200 KB of shared memory.
+static int sort_segments(int group, int maxc, size_t* smem) {
+  int segs = (group + 31) / 32;
+  if (segs > 32) segs = 32;
+  while (segs > 1 && (size_t)(segs + 1) * (maxc + 1) * sizeof(int) > 200 * 1024) --segs;
+  *smem = (size_t)(segs + 1) * (maxc + 1) * sizeof(int);
+  return segs;
+}
+
+static cudaError_t launch_sort(const int* cost, int n, int group, int maxc, int* worklist, cudaStream_t s) {
+  size_t smem = 0;
+  const int segs = sort_segments(group, maxc, &smem);
+  cudaError_t e = cudaFuncSetAttribute(lpt_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  lpt_sort_kernel<<<(n + group - 1) / group, 1024, smem, s>>>(cost, n, group, maxc, segs, worklist);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const int* idx, int cap, int* uni,
@@ -225,8 +271,7 @@ cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const
   quad_union_kernel<<<(unsigned)((items + 3) / 4), 128, (size_t)4 * 4 * words * sizeof(uint32_t), s>>>(
       g, Qn, counts, idx, cap, uni, ucount, useg, qcost, status);
   const int maxc = 2 * ((g.nT + 1) / 2) + 2;
-  lpt_sort_kernel<<<1, 1024, (size_t)(maxc + 1) * sizeof(int), s>>>(qcost, (int)items, (int)items, maxc, worklist);
-  return cudaGetLastError();
+  return launch_sort(qcost, (int)items, (int)items, maxc, worklist, s);
 }
 
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
@@ -241,9 +286,7 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
 cudaError_t launch_rank(const int* key, int n, int max_key, int group, int* worklist, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   if (group <= 0 || group > n) group = n;
-  lpt_sort_kernel<<<(n + group - 1) / group, 1024, (size_t)(max_key + 1) * sizeof(int), s>>>(key, n, group, max_key,
-                                                                                          worklist);
-  return cudaGetLastError();
+  return launch_sort(key, n, group, max_key, worklist, s);
 }
 
 }  // namespace fvattn
