@@ -177,37 +177,56 @@ __device__ inline uint32_t order_key(float v) {
 }
 
 constexpr int kSelWarps = 8;     // rows (warps) per selection block
-constexpr int kMaxRounds = 32;   // argmax rounds before falling back to bisection
+// Argmax rounds before falling back to bisection: a round costs about as
+// much as four bisection steps, so rows whose cut (or k_min floor) lies
+// deeper than this are cheaper to bisect.
+#ifndef FVATTN_SEL_ROUNDS
+#define FVATTN_SEL_ROUNDS 8
+#endif
+constexpr int kMaxRounds = FVATTN_SEL_ROUNDS;
 
-// Selection of one row: src holds the row's nT logits; the probabilities'
-// numerators e_j = exp(s_j - max) go to the warp's shared scratch row srow.
+// Selection of one row: src holds the row's nT logits.  Each lane keeps its
+// tiles' order keys in registers (a tile past nT has key 0, below every
+// logit's key) and the numerators e_j = exp(s_j - max) in the warp's shared
+// scratch row srow; up to 24 values a lane also keeps e_j in registers for
+// the bisection (beyond that the registers would spill).
 template <int MAXV>
 __device__ void select_row(const float* __restrict__ src, float* srow, int nT, float top_p, int k_min,
                            int* count_out, int* list) {
   constexpr int NW = (MAXV + 31) / 32;
+  constexpr bool kEReg = MAXV <= 24;
   const int lane = threadIdx.x & 31;
-  float v[MAXV];
+  uint32_t kv[MAXV];
+  float e[kEReg ? MAXV : 1];
+  float mx = -INFINITY;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int j = i * 32 + lane;
-    v[i] = j < nT ? __ldcs(src + j) : -INFINITY;
+    const float x = j < nT ? __ldcs(src + j) : -INFINITY;
+    kv[i] = __float_as_uint(x);
+    mx = fmaxf(mx, x);
   }
-  float mx = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) mx = fmaxf(mx, v[i]);
   mx = warp_max(mx);
   float zp = 0.f;
   const float mx2 = mx * 1.4426950408889634f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int j = i * 32 + lane;
+    const float s = __uint_as_float(kv[i]);
+    kv[i] = j < nT ? order_key(s) : 0u;
+    float x = 0.f;
     if (j < nT) {
-      float e;
-      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(fmaf(v[i], 1.4426950408889634f, -mx2)));
-      srow[j] = e;
-      zp += e;
+      asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(x) : "f"(fmaf(s, 1.4426950408889634f, -mx2)));
+      srow[j] = x;
+      zp += x;
     }
+    if constexpr (kEReg) e[i] = x;
   }
+  // e_j of this lane's element i (only read for a tile below nT)
+  auto ev = [&](int i) -> float {
+    if constexpr (kEReg) return e[i];
+    else return srow[i * 32 + lane];
+  };
   const float Z = warp_sum(zp);
   __syncwarp();
 
@@ -230,21 +249,21 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
   const int rounds = (floor_k > kMaxRounds) ? 0 : (nT < kMaxRounds ? nT : kMaxRounds);
   for (int r = 0; r < rounds; ++r) {
     if (count >= 0 && picks >= count) break;
-    float bv = -INFINITY;
+    uint32_t bk = 0u;
     int bj = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
       const bool free_i = !((tk[i >> 5] >> (i & 31)) & 1u);
-      if (free_i && v[i] > bv) {
-        bv = v[i];
+      if (free_i && kv[i] > bk) {
+        bk = kv[i];
         bj = i * 32 + lane;
       }
     }
     // warp argmax in two single-instruction reductions: the largest key, then
     // the lowest id holding it (a lane's own ties already went to its lowest id)
     {
-      const uint32_t kmx = __reduce_max_sync(0xffffffffu, order_key(bv));
-      bj = (int)__reduce_min_sync(0xffffffffu, order_key(bv) == kmx ? (uint32_t)bj : 0x7fffffffu);
+      const uint32_t kmx = __reduce_max_sync(0xffffffffu, bk);
+      bj = (int)__reduce_min_sync(0xffffffffu, bk == kmx ? (uint32_t)bj : 0x7fffffffu);
     }
     if (bj == 0x7fffffff) break;
     if ((bj & 31) == lane) {
@@ -285,10 +304,7 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
       const uint32_t cand = u | (1u << b);
       float part = 0.f;
 #pragma unroll
-      for (int i = 0; i < MAXV; ++i) {
-        const int j = i * 32 + lane;
-        part += (j < nT && order_key(v[i]) >= cand) ? srow[j] : 0.f;
-      }
+      for (int i = 0; i < MAXV; ++i) part += kv[i] >= cand ? ev(i) : 0.f;
       if (warp_sum(part) >= target) u = cand;
     }
     float gpart = 0.f;
@@ -296,16 +312,12 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
     float eu = 0.f;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
-      const int j = i * 32 + lane;
-      if (j < nT) {
-        const uint32_t kk = order_key(v[i]);
-        if (kk > u) {
-          gpart += srow[j];
-          ++cgt;
-        } else if (kk == u) {
-          ++ceq;
-          eu = srow[j];
-        }
+      if (kv[i] > u) {
+        gpart += ev(i);
+        ++cgt;
+      } else if (kv[i] == u) {
+        ++ceq;
+        eu = ev(i);
       }
     }
     const float mgt = warp_sum(gpart);
@@ -337,12 +349,12 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
       const uint32_t cand = u2 | (1u << b);
       int c = 0;
 #pragma unroll
-      for (int i = 0; i < MAXV; ++i) c += (i * 32 + lane < nT && order_key(v[i]) >= cand) ? 1 : 0;
+      for (int i = 0; i < MAXV; ++i) c += kv[i] >= cand ? 1 : 0;
       if (warp_isum(c) >= count) u2 = cand;
     }
     int cgt = 0;
 #pragma unroll
-    for (int i = 0; i < MAXV; ++i) cgt += (i * 32 + lane < nT && order_key(v[i]) > u2) ? 1 : 0;
+    for (int i = 0; i < MAXV; ++i) cgt += kv[i] > u2 ? 1 : 0;
     cgt = warp_isum(cgt);
     uT = u2;
     take = count - cgt;
@@ -351,11 +363,11 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int j = i * 32 + lane;
-    const uint32_t kk = j < nT ? order_key(v[i]) : 0u;
-    const bool tie = j < nT && kk == uT;
+    const bool valid = j < nT;
+    const bool tie = valid && kv[i] == uT;
     const unsigned tmask = __ballot_sync(0xffffffffu, tie);
     const int trank = tie_base + __popc(tmask & ((1u << lane) - 1u));
-    const bool sel = j < nT && (kk > uT || (tie && trank < take));
+    const bool sel = valid && (kv[i] > uT || (tie && trank < take));
     const unsigned smask = __ballot_sync(0xffffffffu, sel);
     const int pos = base + __popc(smask & ((1u << lane) - 1u));
     if (sel && pos < count) out[pos] = j;

@@ -58,6 +58,7 @@ namespace ft {
 #ifndef FVATTN_FT_ISSUE
 #define FVATTN_FT_ISSUE 0
 #endif
+
 constexpr int D = 128;
 constexpr int KST = FVATTN_FT_KSTAGES;     // K ring depth
 constexpr int VST = FVATTN_FT_VSTAGES;     // V ring depth
@@ -84,13 +85,13 @@ struct Ctl {
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[SBUF];   // S ready (MMA commit) + step info written (MMA thread arrive)
-  uint64_t p_full[SBUF];   // both halves' P written (256 softmax threads)
+  uint64_t p_full[SBUF];   // both halves' P written (one arrival per softmax warp)
   uint64_t pv_done[SBUF];  // PV of step c complete: barrier c & 1, phase c >> 1 (the S of step
                            // c waits for PV(c - 2), and PV(c + 2) needs P(c + 2), so a waiter
                            // never sees two outstanding phases)
-  uint64_t o_empty;        // epilogue read both O (256 arrivals per item)
-  uint64_t xchg1;          // epilogue: group 1 published (m, l) (128 arrivals per item)
-  uint64_t xchg2;          // epilogue: group 0 replaced them with the merge scales (128 per item)
+  uint64_t o_empty;        // epilogue read both O (8 warp arrivals per item)
+  uint64_t xchg1;          // epilogue: group 1 published (m, l) (4 warp arrivals per item)
+  uint64_t xchg2;          // epilogue: group 0 replaced them with the merge scales (4 per item)
   uint64_t drain;          // final commits of the two MMA threads
   int info[SBUF];          // per S buffer: the step word
   int meta[KST];
@@ -330,12 +331,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     }
     for (int i = 0; i < SBUF; ++i) {
       mbar_init(&ctl->s_full[i], 2);
-      mbar_init(&ctl->p_full[i], 256);
+      mbar_init(&ctl->p_full[i], 8);      // one arrival per softmax warp
       mbar_init(&ctl->pv_done[i], 1);
     }
-    mbar_init(&ctl->o_empty, 256);
-    mbar_init(&ctl->xchg1, 128);
-    mbar_init(&ctl->xchg2, 128);
+    mbar_init(&ctl->o_empty, 8);
+    mbar_init(&ctl->xchg1, 4);
+    mbar_init(&ctl->xchg2, 4);
     mbar_init(&ctl->drain, ISSUE == 2 ? 1 : 2);   // one final commit per MMA issuer
     ctl->abort = 0;
     fence_mbar_init();
@@ -768,7 +769,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ctl->p_full[b]);
+        mbar_arrive_warp(&ctl->p_full[b]);
         ++c;
         if (info & STEP_LAST) break;
       }
@@ -780,7 +781,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       float s0 = 0.f, s1 = 0.f, M = -INFINITY, L = 0.f;
       if (h == 1) {
         ctl->ex[r] = make_float2(m_use, l);
-        mbar_arrive(&ctl->xchg1);
+        mbar_arrive_warp(&ctl->xchg1);
         if (!mbar_wait(&ctl->xchg2, (uint32_t)(k & 1), abort_flag, a.status, cap)) break;
         const float2 sc = ctl->ex[r];
         s0 = sc.x;
@@ -796,7 +797,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         s0 = w0 * inv;
         s1 = w1 * inv;
         ctl->ex[r] = make_float2(s0, s1);
-        mbar_arrive(&ctl->xchg2);
+        mbar_arrive_warp(&ctl->xchg2);
       }
       const int tok = !valid ? 0 : (a.out_nat ? cube_row_token(g, cube, rr) : tile * kTileTokens + rr);
       __nv_bfloat16* orow = a.out + ((size_t)bh * g.N + tok) * D + 64 * h;
@@ -821,7 +822,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       if (valid && h == 0)
         a.lse[(size_t)bh * g.N + tok] = L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
       tc_fence_before();
-      mbar_arrive(&ctl->o_empty);
+      mbar_arrive_warp(&ctl->o_empty);
     }
   }
 
