@@ -14,6 +14,9 @@ Multi-GPU: one process per GPU (torchrun); every rank runs an independent
 replica of the workload (heads shard with no exchange), the time is the max
 over ranks and ``value`` counts the work of all ranks ("scaling": "weak").
 ``--impl reference`` times the CPU oracle on a bounded sample instead.
+A single-GPU line also carries ``secondary``: the same forward, device-timed,
+on the 720p latent (20x48x80 = 76,800 tokens, 3D Hilbert order, RoPE in the
+loads) with its own stage times, roofline and CTA load balance.
 """
 from __future__ import annotations
 
@@ -282,6 +285,66 @@ def run_reference(args, wl):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
+SECONDARY = "wan720p_hilbert_rope"
+
+
+def run_secondary(args, dev, name: str = SECONDARY, steps: int = 5, warmup: int = 3) -> dict:
+    """The forward on a second workload (720p, 3D Hilbert order, RoPE applied in
+    the loads), device-timed like the main line: its own stage times, the
+    fine kernel's roofline, the CTA load balance and the workspace it needs."""
+    import torch
+    from block_sparse_spatiotemporal_b200 import fvattn as F
+    wl = WORKLOADS[name]
+    q, k, v = make_inputs(wl)
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
+    del q, k, v
+    shape = F.make_shape(wl.batch, wl.heads, wl.head_dim, wl.grid, dtype=F.BF16,
+                         order=F.HILBERT if wl.order == "hilbert" else F.RASTER_CUBE)
+    rope = F.make_rope(wl.rope_dims, wl.rope_base) if wl.rope else None
+    ws = F.workspace(shape, rope, device=dev)
+    cache, counts, idx = F.new_cache(shape, device=dev)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        F.forward(shape, qd, kd, vd, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=out, lse=lse)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during the second workload's warm-up")
+    pairs = int(counts.sum().item())
+    flops_step = pairs * pair_flops(wl.head_dim)
+    F.profile_read()
+    F.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    F.profile_enable(False)
+    stages = F.profile_read()
+    imbalance = sm_imbalance(F, shape, ws, rope)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set during the second workload's timed steps")
+    ms = e0.elapsed_time(e1) / steps
+    pk, pk_kind = peaks()
+    fine_ms, fine_n = stages["fine"]
+    achieved = flops_step / (fine_ms / max(fine_n, 1) / 1e3) / 1e12
+    return {"workload": wl.name, "config": workload_config(wl, args), "steps": steps, "warmup": warmup,
+            "ms_per_step": ms, "value": flops_step / (ms / 1e3) / 1e12, "unit": UNIT,
+            "selected_pairs": pairs, "density": pairs / (wl.heads * wl.num_tiles ** 2),
+            "stage_ms": {n: round(v[0] / steps, 4) for n, v in stages.items() if v[1]},
+            "roofline": {"kernel": "fine_tc_kernel", "bound": "tensor", "achieved": achieved,
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                         "peak_source": f"{pk_kind} bf16 burst"},
+            "sm_imbalance": imbalance, "gpu_launches": sum(n for _, n in stages.values()),
+            "workspace_mib": F.workspace_size(shape, rope) / 2 ** 20}
+
 def max_over_ranks(ms: float, device, world: int) -> float:
     """The slowest rank's time: every rank takes part (a collective), so the
     job's time is the max.  A single rank returns its own time."""
@@ -459,6 +522,8 @@ def run_gpu(args, wl):
             "clocks": clocks,
             "e2e": e2e,
         }
+        if world == 1 and not args.no_secondary and not args.subblock and wl.name != SECONDARY:
+            line["secondary"] = run_secondary(args, dev)
         if world == 1 and not args.no_cpu_baseline:
             # the oracle leg: its coarse stage runs on every head and checks the GPU's lists row by row
             lists = None if args.subblock else (counts.cpu().numpy(), idx.cpu().numpy())
@@ -876,6 +941,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="wan480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the 720p Hilbert + RoPE forward the single-GPU line also reports")
     ap.add_argument("--sweep", action="store_true", help="the 480p top-p / top-k / cached-mask sweep (one JSON line)")
     ap.add_argument("--subblock", action="store_true",
                     help="hierarchical sub-block scoring (pool_select_subblock + block_sparse_fwd)")

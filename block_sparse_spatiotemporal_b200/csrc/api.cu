@@ -109,9 +109,8 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   L.useg = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.qcost = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.cta_times = take(sizeof(unsigned long long) * (1 + 2 * (size_t)kMaxCtas));
-  const size_t rot = rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0;
-  L.qrot = take(rot);
-  L.krot = take(rot);
+  // RoPE: the rotated K (tiled); the rotated Q goes to the caller's output buffer
+  L.krot = take(rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0);
   if (sub) {
     const size_t sb = sizeof(float) * (size_t)g.BH * g.nT * kSubBlocks * g.d;
     L.sqh = take(sb);
@@ -395,9 +394,12 @@ int check_blocks(const fvattn_blocks* b, const Geom& g) {
   return FVATTN_OK;
 }
 
-// Pool (+ RoPE) and select into `blocks`; writes rotated copies if asked.
+// Pool (+ RoPE) and select into `blocks`.  qrot (RoPE only): where the
+// rotated Q goes, in the call's layout (the fine stage's output buffer); the
+// rotated K goes to the workspace, tiled.
 int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
-               bool natural, bool pooled, bool rot, float top_p, int k_min, const fvattn_blocks* blocks) {
+               bool natural, bool pooled, void* qrot, float top_p, int k_min, const fvattn_blocks* blocks) {
+  const bool rot = qrot != nullptr;
   const bool r = rope_on(rope);
   PooledOut po{};
   if (pooled) {
@@ -410,7 +412,7 @@ int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const vo
   StageTimer t(FVATTN_STAGE_POOL, c.s);
   FV_CUDA(launch_pool(c.g, shape->dtype, q, k, natural ? 1 : 0, c.at<int>(c.L.tile_cube), c.at<int>(c.L.tile_tok),
                       r ? 1 : 0, r ? rope->dt : 0, r ? rope->dh : 0, r ? rope->dw : 0, c.at<float2>(c.L.rope_tab),
-                      po, rot ? c.at<void>(c.L.qrot) : nullptr, rot ? c.at<void>(c.L.krot) : nullptr, c.s));
+                      po, qrot, rot ? c.at<void>(c.L.krot) : nullptr, c.s));
   t.kernels = 1;
   }
   if (!pooled) return FVATTN_OK;
@@ -476,21 +478,22 @@ int run_schedule_quad(const Call& c, const fvattn_blocks* blocks) {
   return FVATTN_OK;
 }
 
-// Fine stage.  q/k come from the rotated tiled copies when RoPE is on.
+// Fine stage.  Under RoPE, q is the rotated copy the coarse stage wrote into
+// `out` (call layout) and k the rotated tiled copy in the workspace.
 // worklist / grid: a caller's work list and persistent grid (default: the
 // schedule's work list in the workspace and one CTA per SM).
 int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void* k, const void* v,
              const fvattn_rope* rope, bool natural, const fvattn_blocks* blocks, void* out, float* lse,
              const int* worklist = nullptr, int grid = 0) {
   const bool r = rope_on(rope);
-  const void* qs = r ? c.at<void>(c.L.qrot) : q;
+  const void* qs = r ? out : q;
   const void* ks = r ? c.at<void>(c.L.krot) : k;
-  const bool qk_nat = natural && !r;
+  const bool k_nat = natural && !r;
   if (kFineQuad && shape->dtype == FVATTN_BF16 && !worklist) {
     // quad items over the schedule of run_schedule_quad
     CUtensorMap mq, mk, mv;
-    FV_TRY(make_tile_map(&mq, qs, c.g, qk_nat));
-    FV_TRY(make_tile_map(&mk, ks, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mq, qs, c.g, natural));
+    FV_TRY(make_tile_map(&mk, ks, c.g, k_nat));
     FV_TRY(make_tile_map(&mv, v, c.g, natural));
     FineQArgs a{};
     a.g = c.g;
@@ -502,8 +505,8 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.n_items = c.g.BH * c.g.Qn;
     a.Qn = c.g.Qn;
     a.tile_cube = c.at<int>(c.L.tile_cube);
-    a.q_nat = qk_nat;
-    a.k_nat = qk_nat;
+    a.q_nat = natural;
+    a.k_nat = k_nat;
     a.v_nat = natural;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
@@ -516,8 +519,8 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
   } else if (shape->dtype == FVATTN_BF16) {
     // two-tile items over a caller's work list (augmented lists)
     CUtensorMap mq, mk, mv;
-    FV_TRY(make_tile_map(&mq, qs, c.g, qk_nat));
-    FV_TRY(make_tile_map(&mk, ks, c.g, qk_nat));
+    FV_TRY(make_tile_map(&mq, qs, c.g, natural));
+    FV_TRY(make_tile_map(&mk, ks, c.g, k_nat));
     FV_TRY(make_tile_map(&mv, v, c.g, natural));
     FineTcArgs a{};
     a.g = c.g;
@@ -527,8 +530,8 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.worklist = worklist ? worklist : c.at<int>(c.L.worklist);
     a.n_items = c.g.BH * c.g.P;
     a.tile_cube = c.at<int>(c.L.tile_cube);
-    a.q_nat = qk_nat;
-    a.k_nat = qk_nat;
+    a.q_nat = natural;
+    a.k_nat = k_nat;
     a.v_nat = natural;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
@@ -544,8 +547,8 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.q = static_cast<const float*>(qs);
     a.k = static_cast<const float*>(ks);
     a.v = static_cast<const float*>(v);
-    a.q_nat = qk_nat;
-    a.k_nat = qk_nat;
+    a.q_nat = natural;
+    a.k_nat = k_nat;
     a.v_nat = natural;
     a.counts = blocks->counts;
     a.idx = blocks->idx;
@@ -613,7 +616,7 @@ int fvattn_pool_select(const fvattn_shape* shape, const void* q, const void* k, 
   FV_TRY(check_blocks(out, c.g));
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
-  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, false, top_p, k_min, out));
+  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, nullptr, top_p, k_min, out));
   return FVATTN_OK;
 }
 
@@ -684,7 +687,7 @@ int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void
   FV_TRY(check_blocks(blocks, c.g));
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
-  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
+  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, out, 0.f, 0, blocks));
   if (shape->dtype == FVATTN_BF16) FV_TRY(kFineQuad ? run_schedule_quad(c, blocks)
                                                    : run_schedule(c, blocks, c.at<int>(c.L.worklist), shape->dtype,
                                                                   true));
@@ -703,7 +706,7 @@ int fvattn_augment_lists(const fvattn_shape* shape, const void* q, const void* k
   FV_TRY(check_blocks(out, c.g));
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
-  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, false, 0.f, 0, nullptr));
+  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, nullptr, 0.f, 0, nullptr));
   FV_TRY(run_schedule(c, base, worklist));
   const int items = c.g.BH * c.g.P;
   int G = num_ctas > 0 ? num_ctas : c.dev.sms;
@@ -729,7 +732,7 @@ int fvattn_block_sparse_fwd_worklist(const fvattn_shape* shape, const void* q, c
   FV_TRY(check_blocks(blocks, c.g));
   const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
   FV_TRY(tables(c, rope, rope_on(rope) && !natural));
-  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, true, 0.f, 0, blocks));
+  if (rope_on(rope)) FV_TRY(run_coarse(c, shape, q, k, rope, natural, false, out, 0.f, 0, blocks));
   {
     StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
     FV_CUDA(launch_union(c.g, blocks->counts, blocks->idx, blocks->cap, c.at<int>(c.L.uni), c.at<int>(c.L.ucount),
@@ -780,9 +783,9 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
   }
   FV_TRY(tables(c, rope, false));
   if (!reuse_mask) {
-    FV_TRY(run_coarse(c, &sh, q, k, rope, true, true, rope_on(rope), top_p, k_min, blocks));
+    FV_TRY(run_coarse(c, &sh, q, k, rope, true, true, rope_on(rope) ? out : nullptr, top_p, k_min, blocks));
   } else if (rope_on(rope)) {
-    FV_TRY(run_coarse(c, &sh, q, k, rope, true, false, true, 0.f, 0, blocks));
+    FV_TRY(run_coarse(c, &sh, q, k, rope, true, false, out, 0.f, 0, blocks));
   }
   if (sh.dtype == FVATTN_BF16) FV_TRY(kFineQuad ? run_schedule_quad(c, blocks)
                                                : run_schedule(c, blocks, c.at<int>(c.L.worklist), sh.dtype, true));

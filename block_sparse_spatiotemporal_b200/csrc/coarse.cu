@@ -121,7 +121,11 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
 #pragma unroll
     for (int i = 0; i < DPL; ++i) acc[i] += v[it][i];
     if (rot) {
-      T* dst = rot + ((size_t)bh * g.N + (size_t)j * kTileTokens + r) * D + col;
+      // Q: at the position it was read from (the caller's output buffer, whose
+      // rows of this tile the fine stage overwrites only after reading them);
+      // K: tiled, the layout the fine stage streams key tiles in
+      const int n = which == 0 && natural ? cube_row_token(g, cube, r) : j * kTileTokens + r;
+      T* dst = rot + ((size_t)bh * g.N + n) * D + col;
       Vec<T, DPL>::store(dst, v[it]);
     }
   }

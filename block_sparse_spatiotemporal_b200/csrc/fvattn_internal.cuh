@@ -66,7 +66,7 @@ struct WsLayout {
   size_t useg, qcost;    // int32 [BH*Qn] quad items: union segments and cost
   size_t cta_times;      // u64 [1 + 2 * kMaxCtas] fine-stage CTA start / end times (profiling)
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
-  size_t qrot, krot;     // dtype [BH*N*d] rotated copies (rope only)
+  size_t krot;           // dtype [BH*N*d] rotated K, tiled (rope only)
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
   size_t skh, skl;       //   ... of K
   size_t tmass;          //   float [BH*nT*8*nT] log2 key-tile masses per query sub-block

@@ -31,6 +31,10 @@
  * Execution.  Calls enqueue kernels on the given stream and return without
  *   synchronising (except fvattn_get_device_status).  Calls that share a
  *   workspace must not overlap in time.
+ * Outputs.  out must not overlap q, k or v: with RoPE enabled the forward
+ *   calls first write the rotated Q into out (each query row where its
+ *   output row goes) and the fine stage overwrites it with the output; the
+ *   rotated K goes to the workspace.
  * Errors.  Argument, shape and capacity errors are detected on the host and
  *   returned before anything is enqueued.  A failed launch returns
  *   FVATTN_ERR_CUDA.  Errors found by a kernel (an out-of-range block index,
