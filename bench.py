@@ -56,8 +56,11 @@ def peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
+    # the kernel and the work-list order it runs (which decides its L2 reuse)
     for rel in ("block_sparse_spatiotemporal_b200/csrc/fine_tc.cu",
-                "block_sparse_spatiotemporal_b200/csrc/fvattn_internal.cuh"):
+                "block_sparse_spatiotemporal_b200/csrc/fvattn_internal.cuh",
+                "block_sparse_spatiotemporal_b200/csrc/schedule.cu",
+                "block_sparse_spatiotemporal_b200/csrc/api.cu"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

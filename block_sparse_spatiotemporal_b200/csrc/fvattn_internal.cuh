@@ -521,10 +521,10 @@ cudaError_t launch_scores_sub(const CUtensorMap& mqh, const CUtensorMap& mql, co
 cudaError_t launch_subblock_agg(const Geom& g, const float* Tb, float* logp, cudaStream_t s);
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
                          cudaStream_t s);
-// Longest-first order of n items by key (descending; ties by ascending item
-// index), keys in [0, max_key], within each group of `group` consecutive
-// items (group <= 0: one group).
-cudaError_t launch_rank(const int* key, int n, int max_key, int group, int* worklist, cudaStream_t s);
+// Longest-first order of n items by key >> shift (descending; ties by
+// ascending item index), keys in [0, max_key], within each group of `group`
+// consecutive items (group <= 0: one group).
+cudaError_t launch_rank(const int* key, int n, int max_key, int group, int shift, int* worklist, cudaStream_t s);
 cudaError_t launch_fine_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FineTcArgs& a,
                            int num_sms, cudaStream_t s);
 cudaError_t launch_fine_f32(const FineF32Args& a, cudaStream_t s);

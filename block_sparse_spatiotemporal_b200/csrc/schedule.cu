@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(128) quad_union_kernel(Geom g, int Qn, const i
 // places its segment's items 32 at a time in code order (ranks among equal
 // costs from __match_any_sync): stable and deterministic.
 __global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ cost_all, int n_all, int group, int maxc,
-                                                        int segs, int* __restrict__ worklist_all) {
+                                                        int shift, int segs, int* __restrict__ worklist_all) {
   extern __shared__ int sort_smem[];
   int* hist = sort_smem;                         // [segs][maxc + 1]: counts, then running offsets
   int* base = sort_smem + segs * (maxc + 1);     // [maxc + 1]: items of larger cost
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ 
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int i = i0 + u * 32 + lane;
-        cv[u] = i < hi ? min(max(cost[i], 0), maxc) : -1;
+        cv[u] = i < hi ? min(max(cost[i], 0), maxc) >> shift : -1;
       }
 #pragma unroll
       for (int u = 0; u < U; ++u)
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(1024) lpt_sort_kernel(const int* __restrict__ 
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int i = b0 + u * 32 + lane;
-        cv[u] = i < hi ? min(max(cost[i], 0), maxc) : -1;
+        cv[u] = i < hi ? min(max(cost[i], 0), maxc) >> shift : -1;
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -293,12 +293,13 @@ static int sort_segments(int group, int maxc, size_t* smem) {
   return segs;
 }
 
-static cudaError_t launch_sort(const int* cost, int n, int group, int maxc, int* worklist, cudaStream_t s) {
+static cudaError_t launch_sort(const int* cost, int n, int group, int maxc, int shift, int* worklist,
+                               cudaStream_t s) {
   size_t smem = 0;
   const int segs = sort_segments(group, maxc, &smem);
   cudaError_t e = cudaFuncSetAttribute(lpt_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  lpt_sort_kernel<<<(n + group - 1) / group, 1024, smem, s>>>(cost, n, group, maxc, segs, worklist);
+  lpt_sort_kernel<<<(n + group - 1) / group, 1024, smem, s>>>(cost, n, group, maxc, shift, segs, worklist);
   return cudaGetLastError();
 }
 
@@ -310,7 +311,7 @@ cudaError_t launch_quad_schedule(const Geom& g, int Qn, const int* counts, const
   quad_union_kernel<<<(unsigned)((items + 3) / 4), 128, (size_t)4 * 4 * words * sizeof(uint32_t), s>>>(
       g, Qn, counts, idx, cap, uni, ucount, useg, qcost, status);
   const int maxc = 2 * ((g.nT + 1) / 2) + 2;
-  return launch_sort(qcost, (int)items, (int)items, maxc, worklist, s);
+  return launch_sort(qcost, (int)items, (int)items, maxc, 0, worklist, s);
 }
 
 cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int cap, int* uni, int* ucount, int* status,
@@ -324,10 +325,10 @@ cudaError_t launch_union(const Geom& g, const int* counts, const int* idx, int c
   return cudaGetLastError();
 }
 
-cudaError_t launch_rank(const int* key, int n, int max_key, int group, int* worklist, cudaStream_t s) {
+cudaError_t launch_rank(const int* key, int n, int max_key, int group, int shift, int* worklist, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   if (group <= 0 || group > n) group = n;
-  return launch_sort(key, n, group, max_key, worklist, s);
+  return launch_sort(key, n, group, max_key, shift, worklist, s);
 }
 
 }  // namespace fvattn
