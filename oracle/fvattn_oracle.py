@@ -584,7 +584,7 @@ def lpt_order(costs):
     return sorted(range(len(costs)), key=lambda i: (-costs[i], i))
 
 
-def augment_lists(S, counts, idx, num_ctas):
+def augment_lists(S, counts, idx, num_ctas, cta_busy_ns=None, fill_percent=100):
     """Slack-aware augmentation on one GPU ("FVAttn" digest, section 02: ranks
     off the critical path spend their spare time on extra, somewhat
     important blocks), with the persistent fine stage's CTAs as the ranks.
@@ -598,6 +598,14 @@ def augment_lists(S, counts, idx, num_ctas):
     over the item's rows with a list (ties to the lower tile), added to each
     of those rows.  S [BH, nT, nT] are the coarse logits.
 
+    With ``cta_busy_ns`` (one measured busy time per CTA, from a run of the
+    same work list on the unaugmented lists) a CTA's slack is its measured
+    idle time instead, turned into union entries at the run's mean time per
+    entry and scaled by ``fill_percent``:
+    floor((max busy - busy_c) * total entries * fill / (100 * total busy)),
+    in exact integer arithmetic (the spare time the digest's ranks spend is
+    time, which entry counts only approximate).
+
     Returns (counts, idx, extra, worklist): the augmented lists (ascending),
     the tiles added per item, and the work list the fine stage keeps (the
     order of the unaugmented costs)."""
@@ -609,10 +617,17 @@ def augment_lists(S, counts, idx, num_ctas):
     G = max(1, min(num_ctas, len(order)))
     loads = [sum(costs[order[t]] for t in range(c, len(order), G)) for c in range(G)]
     top = max(loads)
+    if cta_busy_ns is not None:
+        busy = [int(b) for b in cta_busy_ns[:G]]
+        total_busy, total_load, top_busy = sum(busy), sum(loads), max(busy)
+        slacks = [((top_busy - b) * total_load * int(fill_percent)) // (100 * total_busy) if total_busy > 0 else 0
+                  for b in busy]
+    else:
+        slacks = [top - ld for ld in loads]
     extra = [0] * len(order)
     for c in range(G):
         slots = list(range(c, len(order), G))
-        slack, n = top - loads[c], len(slots)
+        slack, n = slacks[c], len(slots)
         for u, t in enumerate(slots):
             extra[order[t]] = slack // n + (1 if u < slack % n else 0)
     new_counts = counts.copy()

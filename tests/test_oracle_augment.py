@@ -120,3 +120,48 @@ def test_hand_worked_split_of_the_slack():
     assert added == [0, 2, 0, 1]
     assert i2[0, 2, :c2[0, 2]].tolist() == [0, 1, 3, 4] and i2[0, 3, :c2[0, 3]].tolist() == [2, 3, 4]
     assert i2[0, 6, :c2[0, 6]].tolist() == [6, 7] and i2[0, 7, :c2[0, 7]].tolist() == [6, 7]
+
+
+def _hand_lists():
+    nT = 8
+    counts = np.zeros((1, nT), np.int64)
+    idx = np.zeros((1, nT, nT), np.int64)
+    lists = {0: [0, 1, 2], 1: [3, 4], 2: [0, 1], 3: [2], 4: [5], 5: [6], 6: [7], 7: [7]}
+    for r, lst in lists.items():
+        counts[0, r] = len(lst)
+        idx[0, r, :len(lst)] = lst
+    return counts, idx
+
+
+def test_measured_slack_hand_worked():
+    """The same four items (costs 5, 3, 2, 1; CTA 0 runs items 0 and 2, CTA 1
+    items 1 and 3; 11 union entries in all) with measured busy times.
+    CTA 0 at 500 ns and CTA 1 at 600 ns: CTA 1 is the slower one although it
+    has fewer entries, so CTA 0 gets the slack, (600 - 500) * 11 * 100 /
+    (100 * 1100) = 1 entry, on its first item (item 0, rows 0 and 1, union
+    {0..4}); all logits are equal, so the lowest outside tile, 5, is added to
+    both rows.  At 700 / 400 ns with fill 50%: CTA 1's slack is
+    floor(300 * 11 * 50 / (100 * 1100)) = floor(1.5) = 1, on item 1 (rows 2
+    and 3, union {0, 1, 2}): tile 3 is added to both rows."""
+    counts, idx = _hand_lists()
+    S = np.zeros((1, 8, 8))
+    c2, i2, added, order = O.augment_lists(S, counts, idx, 2, cta_busy_ns=[500, 600])
+    assert order == [0, 1, 2, 3] and added == [1, 0, 0, 0]
+    assert i2[0, 0, :c2[0, 0]].tolist() == [0, 1, 2, 5] and i2[0, 1, :c2[0, 1]].tolist() == [3, 4, 5]
+    assert np.array_equal(c2[0, 2:], counts[0, 2:])
+    c3, i3, added3, _ = O.augment_lists(S, counts, idx, 2, cta_busy_ns=[700, 400], fill_percent=50)
+    assert added3 == [0, 1, 0, 0]
+    assert i3[0, 2, :c3[0, 2]].tolist() == [0, 1, 3] and i3[0, 3, :c3[0, 3]].tolist() == [2, 3]
+
+
+def test_measured_slack_proportional_to_entries_matches_entry_slack():
+    """Busy times proportional to the CTAs' entry loads give back the entry
+    slack exactly; fill 0 adds nothing."""
+    S, counts, idx = _case(BH=4, nT=12, seed=5, density=0.2)
+    for G in (3, 7):
+        c1, i1, added1, order = O.augment_lists(S, counts, idx, G)
+        busy = [1000 * ld for ld in _loads(counts, idx, order, G, 12)]
+        c2, i2, added2, _ = O.augment_lists(S, counts, idx, G, cta_busy_ns=busy)
+        assert added1 == added2 and np.array_equal(c1, c2) and np.array_equal(i1, i2)
+        c3, _, added3, _ = O.augment_lists(S, counts, idx, G, cta_busy_ns=busy, fill_percent=0)
+        assert sum(added3) == 0 and np.array_equal(c3, counts)
