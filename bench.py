@@ -866,8 +866,11 @@ def run_backward(args, wl):
 def run_augment(args, wl):
     """Slack-aware augmentation at the workload's shape: the plain path
     (selection, schedule, fine stage) against selection, augmentation to one
-    CTA per SM and the fine stage on the kept work list; one JSON line with
-    both times, the selected pairs before and after, and the fine-stage times."""
+    CTA per SM and the fine stage on the kept work list; then the kept work
+    list on the plain lists ("kept"), whose last step's per-CTA busy times
+    size a second augmentation ("measured": slack = measured idle time, at
+    --fill percent); one JSON line with every arm's times, the selected pairs
+    and the fine-stage times."""
     import torch
     from block_sparse_spatiotemporal_b200 import fvattn as F
 
@@ -897,29 +900,61 @@ def run_augment(args, wl):
         F.block_sparse_fwd_worklist(shape, qd, kd, vd, aug[0], aug[1], wlist, ws, num_ctas=G, rope=rope,
                                     out=out, lse=lse)
 
-    res = {}
-    for name, fn in (("plain", plain), ("augmented", augmented)):
-        for _ in range(args.warmup):
+    wkept = None      # the kept work list of the plain lists, built before the "kept" arm
+    meas = F.new_blocks(shape, dev)
+    busy_ns = []
+
+    def kept():
+        F.pool_select(shape, qd, kd, ws, wl.top_p, wl.k_min, rope=rope, blocks=base)
+        F.block_sparse_fwd_worklist(shape, qd, kd, vd, base[0], base[1], wkept, ws, num_ctas=G, rope=rope,
+                                    out=out, lse=lse)
+
+    def measured():
+        F.pool_select(shape, qd, kd, ws, wl.top_p, wl.k_min, rope=rope, blocks=base)
+        _, _, wlist = F.augment_lists(shape, qd, kd, ws, base[0], base[1], num_ctas=G, rope=rope,
+                                      out=(meas[0], meas[1]), cta_busy_ns=busy_ns, fill_percent=args.fill)
+        F.block_sparse_fwd_worklist(shape, qd, kd, vd, meas[0], meas[1], wlist, ws, num_ctas=G, rope=rope,
+                                    out=out, lse=lse)
+
+    # the arms alternate step by step (clock and thermal drift fall on all of
+    # them alike); "measured" always follows "kept" and takes its slack from
+    # that step's per-CTA busy times, as a diffusion step would from the last
+    arms = (("plain", plain), ("augmented", augmented), ("kept", kept), ("measured", measured))
+    F.pool_select(shape, qd, kd, ws, wl.top_p, wl.k_min, rope=rope, blocks=base)
+    wkept = F.build_worklist(shape, base[0], base[1], ws)   # the selection is deterministic: same lists each step
+    acc = {name: {"ms": 0.0, "fine": 0.0, "stages": {}} for name, _ in arms}
+    imb = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for step in range(args.warmup + args.steps):
+        for name, fn in arms:
+            if name == "measured":
+                t = F.profile_cta_times(shape, ws, rope)   # the "kept" step just run
+                busy_ns[:] = (t[:, 1] - t[:, 0]).tolist()
+            torch.cuda.synchronize(dev)
+            F.profile_read()
+            F.profile_enable(True)
+            e0.record(stream)
             fn()
-        torch.cuda.synchronize(dev)
-        F.profile_read()
-        F.profile_enable(True)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        F.profile_enable(False)
-        st = F.profile_read()
-        if F.device_status(ws) != 0:
-            raise RuntimeError("device status set")
-        res[name] = {"ms": e0.elapsed_time(e1) / args.steps,
-                     "fine_ms": st["fine"][0] / max(st["fine"][1], 1),
-                     "stage_ms": {k2: round(v2[0] / args.steps, 4) for k2, v2 in st.items() if v2[1]},
-                     "sm_imbalance": sm_imbalance(F, shape, ws, rope)}
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            F.profile_enable(False)
+            st = F.profile_read()
+            if step >= args.warmup:
+                a = acc[name]
+                a["ms"] += e0.elapsed_time(e1)
+                a["fine"] += st["fine"][0]
+                for k2, v2 in st.items():
+                    if v2[1]:
+                        a["stages"][k2] = a["stages"].get(k2, 0.0) + v2[0]
+                imb[name] = sm_imbalance(F, shape, ws, rope)
+    if F.device_status(ws) != 0:
+        raise RuntimeError("device status set")
+    res = {name: {"ms": a["ms"] / args.steps, "fine_ms": a["fine"] / args.steps,
+                  "stage_ms": {k2: round(v2 / args.steps, 4) for k2, v2 in a["stages"].items()},
+                  "sm_imbalance": imb[name]} for name, a in acc.items()}
     pairs = int(base[0].sum().item())
     apairs = int(aug[0].sum().item())
+    mpairs = int(meas[0].sum().item())
     fl = pair_flops(wl.head_dim)
     line = {"metric": "slack-aware augmentation: sparse-attn fwd ms & effective TFLOP/s", "unit": UNIT,
             "value": apairs * fl / (res["augmented"]["ms"] / 1e3) / 1e12, "steps": args.steps,
@@ -927,10 +962,16 @@ def run_augment(args, wl):
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"augment_{wl.name}", "grid": list(wl.grid), "heads": wl.heads,
                        "top_p": wl.top_p, "k_min": wl.k_min, "ctas": G},
-            "selected_pairs": {"plain": pairs, "augmented": apairs, "added": apairs - pairs},
-            "plain": res["plain"], "augmented": res["augmented"],
+            "selected_pairs": {"plain": pairs, "augmented": apairs, "added": apairs - pairs,
+                               "measured": mpairs, "added_measured": mpairs - pairs},
+            "plain": res["plain"], "augmented": res["augmented"], "kept": res["kept"],
+            "measured": dict(res["measured"], fill_percent=args.fill,
+                             extra_fine_vs_kept=res["measured"]["fine_ms"] / res["kept"]["fine_ms"] - 1.0,
+                             added_pairs_frac=(mpairs - pairs) / pairs),
             "fine_tflops": {"plain": pairs * fl / (res["plain"]["fine_ms"] / 1e3) / 1e12,
-                            "augmented": apairs * fl / (res["augmented"]["fine_ms"] / 1e3) / 1e12}}
+                            "augmented": apairs * fl / (res["augmented"]["fine_ms"] / 1e3) / 1e12,
+                            "kept": pairs * fl / (res["kept"]["fine_ms"] / 1e3) / 1e12,
+                            "measured": mpairs * fl / (res["measured"]["fine_ms"] / 1e3) / 1e12}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -956,6 +997,8 @@ def main():
     ap.add_argument("--augment", action="store_true",
                     help="slack-aware augmentation against the plain path at the workload's shape (one JSON line)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--fill", type=int, default=50,
+                    help="--augment: percent of the measured idle time the measured-slack arm fills")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -109,6 +109,7 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   L.useg = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.qcost = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.cta_times = take(sizeof(unsigned long long) * (1 + 2 * (size_t)kMaxCtas));
+  L.cta_busy = take(sizeof(long long) * (size_t)kMaxCtas);
   // RoPE: the rotated K (tiled); the rotated Q goes to the caller's output buffer
   L.krot = take(rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0);
   if (sub) {
@@ -704,26 +705,37 @@ int fvattn_block_sparse_fwd(const fvattn_shape* shape, const void* q, const void
 }
 
 int fvattn_augment_lists(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
-                         const fvattn_blocks* base, int32_t num_ctas, const fvattn_blocks* out, int32_t* worklist,
-                         void* ws, size_t ws_bytes, fvattn_stream_t stream) {
+                         const fvattn_blocks* base, int32_t num_ctas, const int64_t* cta_busy_ns,
+                         int32_t fill_percent, const fvattn_blocks* out, int32_t* worklist, void* ws, size_t ws_bytes,
+                         fvattn_stream_t stream) {
   if (!tensor_ok(q) || !tensor_ok(k) || !worklist || !aligned(worklist, 4)) return FVATTN_ERR_INVALID_ARG;
   if (num_ctas < 0 || num_ctas > 1024) return FVATTN_ERR_INVALID_ARG;
+  if (cta_busy_ns && (fill_percent < 0 || fill_percent > 100)) return FVATTN_ERR_INVALID_ARG;
   Call c;
   FV_TRY(begin(&c, shape, rope, ws, ws_bytes, stream));
   FV_TRY(check_blocks(base, c.g));
   FV_TRY(check_blocks(out, c.g));
-  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
-  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
-  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, nullptr, 0.f, 0, nullptr));
-  FV_TRY(run_schedule(c, base, worklist));
   const int items = c.g.BH * c.g.P;
   int G = num_ctas > 0 ? num_ctas : c.dev.sms;
   if (G > items) G = items;
   if (G > 1024) G = 1024;
+  if (cta_busy_ns)
+    for (int i = 0; i < G; ++i)
+      if (cta_busy_ns[i] < 0 || cta_busy_ns[i] >= (1ll << 40)) return FVATTN_ERR_INVALID_ARG;
+  const bool natural = shape->layout == FVATTN_LAYOUT_NATURAL;
+  FV_TRY(tables(c, rope, rope_on(rope) && !natural));
+  FV_TRY(run_coarse(c, shape, q, k, rope, natural, true, nullptr, 0.f, 0, nullptr));
+  FV_TRY(run_schedule(c, base, worklist));
+  long long* busy = nullptr;
+  if (cta_busy_ns) {
+    busy = c.at<long long>(c.L.cta_busy);
+    FV_CUDA(cudaMemcpyAsync(busy, cta_busy_ns, sizeof(long long) * (size_t)G, cudaMemcpyHostToDevice, c.s));
+  }
   StageTimer t(FVATTN_STAGE_SCHEDULE, c.s);
   // the rank buffer is free once the work list is built: it holds the per-item extra tiles
   FV_CUDA(launch_augment(c.g, c.at<float>(c.L.scores), base->counts, base->idx, base->cap, c.at<int>(c.L.ucount),
-                         worklist, G, c.at<int>(c.L.rank), out->counts, out->idx, out->cap, c.status, c.s));
+                         worklist, G, busy, fill_percent, c.at<int>(c.L.rank), out->counts, out->idx, out->cap,
+                         c.status, c.s));
   t.kernels = 2;
   return FVATTN_OK;
 }

@@ -14,21 +14,46 @@ namespace fvattn {
 
 // One block: load of each CTA over its slots, the largest load, and each
 // item's share of its CTA's slack (the first items in slot order take the
-// remainder).
+// remainder).  With measured busy times (ns, one per CTA, from a run of the
+// same work list on the unaugmented lists) the slack is the CTA's idle time
+// in entries at the run's mean time per entry, times fill_percent / 100:
+// floor((max busy - busy) * total entries * fill / (100 * total busy)),
+// exact in 128-bit integers.
 __global__ void __launch_bounds__(1024) slack_kernel(const int* __restrict__ ucount, const int* __restrict__ worklist,
-                                                     int n_items, int G, int* __restrict__ extra) {
+                                                     int n_items, int G, const long long* __restrict__ busy,
+                                                     int fill_percent, int* __restrict__ extra) {
   __shared__ int top;
-  if (threadIdx.x == 0) top = 0;
+  __shared__ unsigned long long total_load, total_busy, top_busy;
+  if (threadIdx.x == 0) {
+    top = 0;
+    total_load = total_busy = top_busy = 0ull;
+  }
   __syncthreads();
   const int c = threadIdx.x;
   int load = 0, n = 0;
+  long long b = 0;
   if (c < G) {
     for (int t = c; t < n_items; t += G, ++n) load += ucount[worklist[t]];
     atomicMax(&top, load);
+    if (busy) {
+      b = busy[c];
+      atomicAdd(&total_load, (unsigned long long)load);
+      atomicAdd(&total_busy, (unsigned long long)b);
+      atomicMax(&top_busy, (unsigned long long)b);
+    }
   }
   __syncthreads();
   if (c < G) {
-    const int slack = top - load;
+    int slack = top - load;
+    if (busy) {
+      slack = 0;
+      if (total_busy > 0) {
+        const unsigned __int128 num =
+            (unsigned __int128)(top_busy - (unsigned long long)b) * total_load * (unsigned)fill_percent;
+        // at most the total entries: top_busy - b <= total_busy and fill <= 100
+        slack = (int)(num / ((unsigned __int128)100 * total_busy));
+      }
+    }
     int u = 0;
     for (int t = c; t < n_items; t += G, ++u) extra[worklist[t]] = slack / n + (u < slack % n ? 1 : 0);
   }
@@ -131,10 +156,10 @@ __global__ void __launch_bounds__(kAugWarps * 32)
 }
 
 cudaError_t launch_augment(const Geom& g, const float* S, const int* counts, const int* idx, int cap,
-                           const int* ucount, const int* worklist, int G, int* extra, int* out_counts, int* out_idx,
-                           int out_cap, int* status, cudaStream_t s) {
+                           const int* ucount, const int* worklist, int G, const long long* busy, int fill_percent,
+                           int* extra, int* out_counts, int* out_idx, int out_cap, int* status, cudaStream_t s) {
   const int items = g.BH * g.P;
-  slack_kernel<<<1, 1024, 0, s>>>(ucount, worklist, items, G, extra);
+  slack_kernel<<<1, 1024, 0, s>>>(ucount, worklist, items, G, busy, fill_percent, extra);
   const int words = (g.nT + 31) / 32;
   const size_t smem = sizeof(uint32_t) * 4 * words * kAugWarps;
   augment_kernel<<<(items + kAugWarps - 1) / kAugWarps, kAugWarps * 32, smem, s>>>(g, S, counts, idx, cap, extra,

@@ -65,6 +65,7 @@ struct WsLayout {
   size_t worklist;       // int32 [BH*P]
   size_t useg, qcost;    // int32 [BH*Qn] quad items: union segments and cost
   size_t cta_times;      // u64 [1 + 2 * kMaxCtas] fine-stage CTA start / end times (profiling)
+  size_t cta_busy;       // i64 [kMaxCtas] measured CTA busy times for the augmentation's slack
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t krot;           // dtype [BH*N*d] rotated K, tiled (rope only)
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
@@ -549,8 +550,8 @@ cudaError_t launch_key_union(const Geom& g, const int* counts, const int* idx, i
 cudaError_t launch_bwd(const CUtensorMap& s0, const CUtensorMap& s1, const CUtensorMap& m0, const CUtensorMap& m1,
                        const BwdArgs& a, bool key_stationary, int num_sms, cudaStream_t s);
 cudaError_t launch_augment(const Geom& g, const float* S, const int* counts, const int* idx, int cap,
-                           const int* ucount, const int* worklist, int G, int* extra, int* out_counts, int* out_idx,
-                           int out_cap, int* status, cudaStream_t s);
+                           const int* ucount, const int* worklist, int G, const long long* busy, int fill_percent,
+                           int* extra, int* out_counts, int* out_idx, int out_cap, int* status, cudaStream_t s);
 cudaError_t launch_wait_selftest(int* status, long long cap, cudaStream_t s);
 
 }  // namespace fvattn

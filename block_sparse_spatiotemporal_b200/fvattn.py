@@ -101,8 +101,9 @@ _SIGS = {
                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                        ctypes.c_void_p],
     "fvattn_augment_lists": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(Rope),
-                             ctypes.POINTER(Blocks), ctypes.c_int32, ctypes.POINTER(Blocks), ctypes.c_void_p,
-                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p],
+                             ctypes.POINTER(Blocks), ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                             ctypes.POINTER(Blocks), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                             ctypes.c_void_p],
     "fvattn_block_sparse_fwd_worklist": [ctypes.POINTER(Shape), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.POINTER(Rope), ctypes.POINTER(Blocks), ctypes.c_void_p,
                                          ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -323,9 +324,11 @@ def forward(shape: Shape, q, k, v, ws, top_p: float, k_min: int, rope: Optional[
 
 
 def augment_lists(shape: Shape, q, k, ws, counts, idx, num_ctas: int = 0, rope: Optional[Rope] = None, out=None,
-                  stream=None):
+                  stream=None, cta_busy_ns=None, fill_percent: int = 100):
     """Slack-aware augmentation of (counts, idx): returns (counts, idx,
-    worklist) -- the augmented lists and the work list to run them with."""
+    worklist) -- the augmented lists and the work list to run them with.
+    cta_busy_ns: None, or one measured busy time (ns) per CTA of a run of the
+    same work list on the unaugmented lists (a host sequence of ints)."""
     if out is None:
         oc, oi, ob = new_blocks(shape, q.device)
     else:
@@ -333,10 +336,14 @@ def augment_lists(shape: Shape, q, k, ws, counts, idx, num_ctas: int = 0, rope: 
         ob = _blocks_of(oc, oi)
     wl = torch.empty(shape.batch * shape.heads * ((num_tiles(shape) + 1) // 2), dtype=torch.int32, device=q.device)
     base = _blocks_of(counts, idx)
+    busy = None
+    if cta_busy_ns is not None:
+        vals = [int(x) for x in cta_busy_ns]
+        busy = (ctypes.c_int64 * max(1, len(vals)))(*vals)
     _check("fvattn_augment_lists",
            lib().fvattn_augment_lists(ctypes.byref(shape), _ptr(q), _ptr(k), _rope_ptr(rope), ctypes.byref(base),
-                                      int(num_ctas), ctypes.byref(ob), _ptr(wl), _ptr(ws), ws.numel(),
-                                      _stream(stream)))
+                                      int(num_ctas), busy, int(fill_percent), ctypes.byref(ob), _ptr(wl), _ptr(ws),
+                                      ws.numel(), _stream(stream)))
     return oc, oi, wl
 
 

@@ -242,10 +242,19 @@ int fvattn_forward(const fvattn_shape* shape, const void* q, const void* k, cons
  * `base` itself.  Run the fine stage with fvattn_block_sparse_fwd_worklist
  * and the same worklist and num_ctas so that the critical path keeps its
  * length.  num_ctas in [0, 1024], 0 = the device's SM count (the fine
- * stage's grid). */
+ * stage's grid).
+ * cta_busy_ns: NULL (slack in union entries, as above), or a HOST array of
+ *   G = min(num_ctas or the SM count, B*H*P, 1024) busy times in ns, one per
+ *   CTA, each in [0, 2^40), measured on a run of the same work list and
+ *   num_ctas on the unaugmented lists (fvattn_profile_cta_times: end minus
+ *   start).  A CTA's slack is then its measured idle time in entries at that
+ *   run's mean time per entry, scaled by fill_percent in [0, 100]:
+ *   floor((max busy - busy_c) * total entries * fill / (100 * total busy)).
+ *   The array is read during the call. */
 int fvattn_augment_lists(const fvattn_shape* shape, const void* q, const void* k, const fvattn_rope* rope,
-                         const fvattn_blocks* base, int32_t num_ctas, const fvattn_blocks* out,
-                         int32_t* worklist, void* ws, size_t ws_bytes, fvattn_stream_t stream);
+                         const fvattn_blocks* base, int32_t num_ctas, const int64_t* cta_busy_ns,
+                         int32_t fill_percent, const fvattn_blocks* out, int32_t* worklist, void* ws,
+                         size_t ws_bytes, fvattn_stream_t stream);
 
 /* Step 6 with a caller's work list (B*H*P item codes, each once) and
  * persistent grid of num_ctas CTAs (0 = the SM count); otherwise as

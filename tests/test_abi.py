@@ -159,11 +159,15 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
     assert lib.fvattn_block_sparse_bwd(ctypes.byref(f32), *args) == -3
     assert lib.fvattn_block_sparse_bwd(ctypes.byref(s), al, al, al, al, al, al, ctypes.byref(b), None, al, al, al,
                                        1 << 30, None) == -1
-    # augmentation: more than 1024 CTAs, null work list
-    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 2048, ctypes.byref(b), al, al,
-                                    1 << 30, None) == -1
-    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 0, ctypes.byref(b), None, al,
-                                    1 << 30, None) == -1
+    # augmentation: more than 1024 CTAs, null work list, fill outside [0, 100] with measured busy times
+    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 2048, None, 100,
+                                    ctypes.byref(b), al, al, 1 << 30, None) == -1
+    assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 0, None, 100,
+                                    ctypes.byref(b), None, al, 1 << 30, None) == -1
+    busy = (ctypes.c_int64 * 4)(1, 2, 3, 4)
+    for fill in (-1, 101):
+        assert lib.fvattn_augment_lists(ctypes.byref(s), al, al, None, ctypes.byref(b), 4, busy, fill,
+                                        ctypes.byref(b), al, al, 1 << 30, None) == -1
     assert lib.fvattn_block_sparse_fwd_worklist(ctypes.byref(s), al, al, al, None, ctypes.byref(b), None, 0, al, al,
                                                 al, 1 << 30, None) == -1
     # workspace sizes of the new entry points

@@ -30,9 +30,9 @@ def base_lists(wl, q, k, top_p, k_min):
     return counts, idx, S, tol
 
 
-def compare(wl, counts, idx, S, tol, G, gc, gi, gw):
+def compare(wl, counts, idx, S, tol, G, gc, gi, gw, busy=None, fill=100):
     nT, P = wl.num_tiles, (wl.num_tiles + 1) // 2
-    oc, oi, added, order = O.augment_lists(S, counts, idx, G)
+    oc, oi, added, order = O.augment_lists(S, counts, idx, G, cta_busy_ns=busy, fill_percent=fill)
     assert np.array_equal(gw, np.array(order)), "work list"
     unions = O.item_unions(counts, idx, nT)
     ties = 0
@@ -57,6 +57,8 @@ def compare(wl, counts, idx, S, tol, G, gc, gi, gw):
             worst_in = min(score[j] for j in g_add)
             best_out = max([score[j] for j in score if j not in g_add], default=-np.inf)
             assert worst_in >= best_out - t, (item, worst_in, best_out)
+    if busy is not None:      # slack from measured time: the entry loads may move either way
+        return oc, oi, ties
     # the kept work list's critical path did not grow
     costs_b = [max(1, len(x)) for x in unions]
     costs_a = [max(1, len(x)) for x in O.item_unions(gc[0], gi[0], nT)]
@@ -97,6 +99,31 @@ def test_augment_small(case):
                              rope=oracle_rope(wl), blocks=(oc[h], oi[h]))
         assert_close(got[h], ref["out"], "bf16", f"out h{h}")
         assert_close(glse[h], ref["lse"], "bf16", f"lse h{h}")
+
+
+@pytest.mark.parametrize("G,fill", [(16, 100), (16, 37), (5, 0), (200, 60)])
+def test_augment_measured_slack(G, fill):
+    """Slack from per-CTA busy times (seeded synthetic nanoseconds, the same
+    array on both sides) instead of entry counts: work list exact, the same
+    tiles added per item as the oracle's."""
+    wl = Workload("aug", (8, 16, 24), 4, 128, "bf16", 23, 0.85, 2, "raster", False, "per_head")
+    q, k, v = make_inputs(wl)
+    counts, idx, S, tol = base_lists(wl, q, k, wl.top_p, wl.k_min)
+    items = wl.heads * ((wl.num_tiles + 1) // 2)
+    Gc = min(G, items)
+    busy = np.random.default_rng(G * 1000 + fill).integers(1_000_000, 3_000_000, Gc).tolist()
+    shape = shape_of(wl)
+    ws = F.workspace(shape)
+    qd, kd = to_dev(q, "bf16"), to_dev(k, "bf16")
+    cd = torch.from_numpy(counts[None]).cuda()
+    idd = torch.from_numpy(idx[None]).cuda()
+    ac, ai, wlist = F.augment_lists(shape, qd, kd, ws, cd, idd, num_ctas=G, cta_busy_ns=busy, fill_percent=fill)
+    assert F.device_status(ws) == 0
+    gc, gi, gw = ac.cpu().numpy(), ai.cpu().numpy(), wlist.cpu().numpy()
+    _, _, ties = compare(wl, counts, idx, S, tol, Gc, gc, gi, gw, busy=busy, fill=fill)
+    assert ties == 0
+    if fill == 0:
+        assert np.array_equal(gc[0], counts)
 
 
 def test_augment_480p_full():
