@@ -392,12 +392,13 @@ def run_gpu(args, wl):
     lse = torch.empty(qd.shape[:-1], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(qx=qd, kx=kd, vx=vd):
+    def step(qx=qd, kx=kd, vx=vd, o=None):
+        o = out if o is None else o
         if args.subblock:   # sub-block scoring, then the fine stage on its lists
             F.pool_select_subblock(shape, qx, kx, ws, wl.top_p, wl.k_min, rope=rope, blocks=(counts, idx, cache.blocks))
-            F.block_sparse_fwd(shape, qx, kx, vx, counts, idx, ws, rope=rope, out=out, lse=lse)
+            F.block_sparse_fwd(shape, qx, kx, vx, counts, idx, ws, rope=rope, out=o, lse=lse)
         else:
-            F.forward(shape, qx, kx, vx, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=out, lse=lse)
+            F.forward(shape, qx, kx, vx, ws, wl.top_p, wl.k_min, rope=rope, cache=cache, out=o, lse=lse)
 
     for _ in range(max(args.warmup, 1)):
         step()
@@ -434,33 +435,59 @@ def run_gpu(args, wl):
         raise RuntimeError("device status set during the timed region")
     ms_max = max_over_ranks(ms, dev, world)
 
-    # ---- end to end through the public API: pinned host in, host out
+    # ---- end to end through the public API: pinned host in, host out.  A
+    # serving loop's pipeline: step i's inputs go up on one copy stream while
+    # step i-1 computes and step i-2's output comes down on another (PCIe is
+    # full duplex); device inputs and outputs are double-buffered, and events
+    # keep a buffer from being refilled before the step reading it is done.
     e2e = None
     if not args.no_e2e:
         qh, kh, vh = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        qb, kb, vb = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-        for _ in range(2):
-            qb.copy_(qh, non_blocking=True); kb.copy_(kh, non_blocking=True); vb.copy_(vh, non_blocking=True)
-            step(qb, kb, vb)
-            oh.copy_(out, non_blocking=True)
+        ohs = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        ins = [(torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)) for _ in range(2)]
+        outs = [torch.empty_like(out) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+        def pipelined(n):
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(s_in)
+            for i in range(n):
+                b = i % 2
+                if i >= 2:
+                    s_in.wait_event(ev_comp[b])       # step i-2 has read ins[b]
+                with torch.cuda.stream(s_in):
+                    for dst, src in zip(ins[b], (qh, kh, vh)):
+                        dst.copy_(src, non_blocking=True)
+                ev_in[b].record(s_in)
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])      # step i-2's output has left outs[b]
+                step(*ins[b], o=outs[b])
+                ev_comp[b].record(stream)
+                s_out.wait_event(ev_comp[b])
+                with torch.cuda.stream(s_out):
+                    ohs[b].copy_(outs[b], non_blocking=True)
+                ev_out[b].record(s_out)
+            t1.record(s_out)
+            return t0, t1
+
+        pipelined(3)
+        torch.cuda.synchronize(dev)
         n_e2e = max(3, min(args.steps, 20))
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(n_e2e):
-            qb.copy_(qh, non_blocking=True); kb.copy_(kh, non_blocking=True); vb.copy_(vh, non_blocking=True)
-            step(qb, kb, vb)
-            oh.copy_(out, non_blocking=True)
-        s1.record(stream)
+        s0, s1 = pipelined(n_e2e)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(s0.elapsed_time(s1) / n_e2e, dev, world)
         h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
-        d2h = oh.numel() * oh.element_size()
+        d2h = ohs[0].numel() * ohs[0].element_size()
         e2e = {"value": whole_job_value(world, flops_step, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipeline": "inputs of step i up (copy stream) while step i-1 computes and step i-2's output "
+                           "comes down (second copy stream); double-buffered device inputs and outputs"}
+        del ins, outs
 
     # ---- the tile reorder as its own pass (the forward folds it into its loads): q, k, v to
     # tiled layout and out back, 2 bytes moved per byte
