@@ -20,8 +20,8 @@
 
 // 32 MiB.  A shape is accepted when its full workspace
 // (fvattn_workspace_size) fits: for example the 16x32x32 latent with 12
-// heads (13.6 MiB) or the 20x32x52 latent with up to 8 heads (28.9 MiB); the
-// 20x32x52 latent with 9 heads (32.5 MiB) or 40 heads (144.1 MiB) is
+// heads (13.6 MiB) or the 20x32x52 latent with up to 8 heads (29.0 MiB); the
+// 20x32x52 latent with 9 heads (32.6 MiB) or 40 heads (144.2 MiB) is
 // rejected.  The first 4 bytes hold the status word that kernels set on a
 // device-detected error (fvattn_pool_select_noalloc_status reads it).
 static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
