@@ -158,9 +158,10 @@ __global__ void __launch_bounds__(128) pool_kernel(Geom g, const T* __restrict__
 // (element i of a lane is tile 32 i + lane).  Most rows are settled by a few
 // argmax rounds that pick tiles in rank order and add their probabilities in
 // that order until the cut and the k_min floor are both reached.  Rows whose
-// cut lies deeper use a bisection over the 32-bit order-preserving keys of
-// the logits: the largest key u whose suffix mass sum_{key >= u} e reaches
-// top_p * Z (warp-tree sums), then ties at u are taken lowest id first.
+// cut lies deeper search the 32-bit order-preserving keys of the logits for
+// the largest key u whose suffix mass sum_{key >= u} e reaches top_p * Z
+// (warp-tree sums): a bisection of its 16 high bits, then the few keys that
+// share them in descending order; ties at u are taken lowest id first.
 // --------------------------------------------------------------------------
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -188,6 +189,7 @@ constexpr int kSelWarps = 8;     // rows (warps) per selection block
 #define FVATTN_SEL_ROUNDS 8
 #endif
 constexpr int kMaxRounds = FVATTN_SEL_ROUNDS;
+constexpr int kCutRounds = 8;    // distinct keys below the bisected 16-bit prefix taken one by one
 
 // Selection of one row: src holds the row's nT logits.  Each lane keeps its
 // tiles' order keys in registers (a tile past nT has key 0, below every
@@ -303,13 +305,54 @@ __device__ void select_row(const float* __restrict__ src, float* srow, int nT, f
   uint32_t uT = 0;
   int take = 0;
   if (m == 0) {
+    // the cut key u: the largest key whose suffix mass reaches the target.
+    // Its 16 high bits (sign, exponent, 7 mantissa bits) by bisection over
+    // every value ...
     uint32_t u = 0;
-    for (int b = 31; b >= 0; --b) {
+    for (int b = 31; b >= 16; --b) {
       const uint32_t cand = u | (1u << b);
       float part = 0.f;
 #pragma unroll
       for (int i = 0; i < MAXV; ++i) part += kv[i] >= cand ? ev(i) : 0.f;
       if (warp_sum(part) >= target) u = cand;
+    }
+    // ... the rest from the few values sharing them: their distinct keys in
+    // descending order, each adding its values' mass to the mass above the
+    // prefix, until the target is reached (a bisection of the low bits over
+    // every value if that takes more than kCutRounds keys)
+    const uint32_t pre = u >> 16;
+    float above = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) above += (kv[i] >> 16) > pre ? ev(i) : 0.f;
+    const float m_above = warp_sum(above);
+    float acc = 0.f;
+    uint32_t ub = 0xffffffffu;           // keys already added are >= ub
+    bool found = false;
+    for (int rr = 0; rr < kCutRounds && !found; ++rr) {
+      uint32_t bk = 0u;
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i)
+        if ((kv[i] >> 16) == pre && kv[i] < ub && kv[i] > bk) bk = kv[i];
+      const uint32_t kmx = __reduce_max_sync(0xffffffffu, bk);
+      if (kmx == 0u) break;
+      float grp = 0.f;
+#pragma unroll
+      for (int i = 0; i < MAXV; ++i) grp += kv[i] == kmx ? ev(i) : 0.f;
+      acc += warp_sum(grp);
+      if (m_above + acc >= target) {
+        u = kmx;
+        found = true;
+      }
+      ub = kmx;
+    }
+    if (!found) {
+      for (int b = 15; b >= 0; --b) {
+        const uint32_t cand = u | (1u << b);
+        float part = 0.f;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) part += kv[i] >= cand ? ev(i) : 0.f;
+        if (warp_sum(part) >= target) u = cand;
+      }
     }
     float gpart = 0.f;
     int cgt = 0, ceq = 0;
