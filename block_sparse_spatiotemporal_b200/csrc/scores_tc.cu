@@ -9,11 +9,15 @@
 // dropped lo.lo term is below 2^-22 |q||k| per dimension.  The result has
 // about the accuracy of an fp32 FFMA dot product.
 //
-// One CTA per (128 query rows, head), 192 threads: warp 0 loads the CTA's
-// pooled query rows once and streams pooled key rows in 32-dim slices of 128
-// rows (TMA, 3-stage ring); warp 1 issues the MMAs (M=128, N=128, K=8) into
-// one of two TMEM accumulators; warps 2-5 drain a finished 128 x 128 block
-// (thread r = query row r) while the next block is computed.
+// Persistent, one CTA per SM, 192 threads.  A unit is one 128 x 128 block
+// (head, query block, key block); CTA c takes the units [c U / G, (c+1) U / G)
+// of the U in that order, so every CTA gets the same number of blocks within
+// one and consecutive units share their query rows.  Warp 0 loads a unit's
+// pooled query rows when they change (after the MMAs reading the previous
+// ones completed) and streams pooled key rows in 32-dim slices of 128 rows
+// (TMA, 3-stage ring); warp 1 issues the MMAs (M=128, N=128, K=8) into one of
+// two TMEM accumulators; warps 2-5 drain a finished block (thread r = query
+// row r) while the next is computed.
 //
 // Two epilogues.  Tile scores (rows = tiles): the scaled logits go to the
 // fp32 score buffer.  Sub-block scores ("DFSAttn" digest, section 2; rows =
@@ -36,7 +40,7 @@ constexpr uint32_t IDESC = (1u << 4)          // D: f32
                            | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 struct Ctl {
-  uint64_t a_full;
+  uint64_t a_full, a_empty;
   uint64_t b_full[STAGES], b_empty[STAGES];
   uint64_t s_full[2], s_empty[2];
   uint64_t drain;
@@ -81,13 +85,15 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
   __shared__ Ctl ctl;
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rb = blockIdx.x, bh = blockIdx.y;
   const int rows = SUB ? g.nT * kSubBlocks : g.nT;   // pooled rows per head (query and key alike)
-  const int nkc = (rows + 127) / 128;
+  const int nkc = (rows + 127) / 128;                 // 128-row blocks per head
+  const long long units = (long long)g.BH * nkc * nkc;
+  const long long u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
   const long long cap = a.wait_cap;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.a_full, 1);
+    mbar_init(&ctl.a_empty, 1);
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&ctl.b_full[i], 1);
       mbar_init(&ctl.b_empty[i], 1);
@@ -111,13 +117,23 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA
-    mbar_arrive_expect_tx(&ctl.a_full, 2 * DC * BOX);
-    for (int c = 0; c < DC; ++c) {
-      tma_load_3d(sA + c * BOX, &mqh, &ctl.a_full, c * 32, rb * 128, bh);
-      tma_load_3d(sA + (DC + c) * BOX, &mql, &ctl.a_full, c * 32, rb * 128, bh);
-    }
-    int step = 0;
-    for (int j = 0; j < nkc; ++j) {
+    int step = 0, gq = 0;          // key slices issued, query-row groups loaded
+    long long prev = -1;           // bh * nkc + query block of the loaded rows
+    for (long long u = u0; u < u1; ++u) {
+      const long long qg = u / nkc;
+      const int j = (int)(u % nkc), bh = (int)(qg / nkc), rb = (int)(qg % nkc);
+      if (qg != prev) {
+        // the MMAs that read the previous query rows have completed
+        if (gq >= 1 && !mbar_wait(&ctl.a_empty, (uint32_t)(gq - 1) & 1, abort_flag, a.status, cap))
+          goto producer_done;
+        mbar_arrive_expect_tx(&ctl.a_full, 2 * DC * BOX);
+        for (int c = 0; c < DC; ++c) {
+          tma_load_3d(sA + c * BOX, &mqh, &ctl.a_full, c * 32, rb * 128, bh);
+          tma_load_3d(sA + (DC + c) * BOX, &mql, &ctl.a_full, c * 32, rb * 128, bh);
+        }
+        ++gq;
+        prev = qg;
+      }
       for (int c = 0; c < DC; ++c, ++step) {
         const int st = step % STAGES;
         if (step >= STAGES &&
@@ -130,21 +146,30 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
     }
   producer_done:
     // every copy issued has landed before the block exits
-    mbar_drain(&ctl.a_full, 0, a.status, cap);
+    if (gq > 0) mbar_drain(&ctl.a_full, (uint32_t)(gq - 1) & 1, a.status, cap);
     for (int st = 0; st < STAGES && st < step; ++st) {
       const int last = st + ((step - 1 - st) / STAGES) * STAGES;
       mbar_drain(&ctl.b_full[st], (uint32_t)(last / STAGES) & 1, a.status, cap);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA
-    if (mbar_wait(&ctl.a_full, 0, abort_flag, a.status, cap)) {
+    {
       const uint64_t ad0 = umma_desc_sw128(smem_u32(sA), 16, 1024);
       const uint64_t bd0 = umma_desc_sw128(smem_u32(sB), 16, 1024);
-      int step = 0;
+      int step = 0, k = 0, gq = 0;
+      long long prev = -1;
       bool ok = true;
-      for (int j = 0; j < nkc && ok; ++j) {
-        const int b = j & 1;
-        if (j >= 2 && !mbar_wait(&ctl.s_empty[b], (uint32_t)((j >> 1) - 1) & 1, abort_flag, a.status, cap)) break;
+      for (long long u = u0; u < u1 && ok; ++u, ++k) {
+        const long long qg = u / nkc;
+        if (qg != prev) {
+          // the MMAs issued so far read the previous query rows: release them on completion
+          if (gq >= 1) mma_commit(&ctl.a_empty);
+          if (!mbar_wait(&ctl.a_full, (uint32_t)gq & 1, abort_flag, a.status, cap)) break;
+          ++gq;
+          prev = qg;
+        }
+        const int b = k & 1;
+        if (k >= 2 && !mbar_wait(&ctl.s_empty[b], (uint32_t)((k >> 1) - 1) & 1, abort_flag, a.status, cap)) break;
         const uint32_t tS = tbase + 128 * b;
         for (int c = 0; c < DC; ++c, ++step) {
           const int st = step % STAGES;
@@ -176,13 +201,16 @@ __global__ void __launch_bounds__(sc::THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q4 = warp & 3;
     const int row = 32 * q4 + lane;
-    const int grow = rb * 128 + row;
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    float* srow = a.S + ((size_t)bh * rows + (grow < rows ? grow : 0)) * g.nT;
     const float sl2 = g.scale * 1.4426950408889634f;
-    for (int j = 0; j < nkc; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&ctl.s_full[b], (uint32_t)(j >> 1) & 1, abort_flag, a.status, cap)) break;
+    int k = 0;
+    for (long long u = u0; u < u1; ++u, ++k) {
+      const long long qg = u / nkc;
+      const int j = (int)(u % nkc), bh = (int)(qg / nkc), rb = (int)(qg % nkc);
+      const int grow = rb * 128 + row;
+      float* srow = a.S + ((size_t)bh * rows + (grow < rows ? grow : 0)) * g.nT;
+      const int b = k & 1;
+      if (!mbar_wait(&ctl.s_full[b], (uint32_t)(k >> 1) & 1, abort_flag, a.status, cap)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -248,7 +276,15 @@ static cudaError_t launch_scores_t(const CUtensorMap& mqh, const CUtensorMap& mq
       cudaFuncSetAttribute(score_tc_kernel<SUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int rows = SUB ? a.g.nT * kSubBlocks : a.g.nT;
-  dim3 grid((rows + 127) / 128, a.g.BH);
+  const long long nkc = (rows + 127) / 128;
+  const long long units = (long long)a.g.BH * nkc * nkc;
+  if (units <= 0) return cudaSuccess;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(units < sms ? units : sms);   // one CTA per SM (shared memory)
   score_tc_kernel<SUB><<<grid, sc::THREADS, smem, s>>>(mqh, mql, mkh, mkl, a);
   return cudaGetLastError();
 }
