@@ -538,6 +538,9 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.ucount = c.at<int>(c.L.ucount);
     a.worklist = worklist ? worklist : c.at<int>(c.L.worklist);
     a.n_items = c.g.BH * c.g.P;
+    // the schedule's own list runs serpentine; a caller's list (the augmentation's
+    // kept work list, whose per-CTA loads assume CTA c runs c, c + G, ...) does not
+    a.snake = worklist ? 0 : 1;
     a.tile_cube = c.at<int>(c.L.tile_cube);
     a.q_nat = natural;
     a.k_nat = k_nat;

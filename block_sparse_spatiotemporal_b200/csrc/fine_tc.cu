@@ -300,6 +300,16 @@ __device__ __forceinline__ void pv_mmas(uint32_t tbase, uint32_t tP, const uint8
   }
 }
 
+// Work-list slot of this CTA's k-th item: round k of G consecutive slots,
+// CTA c taking slot c of each round, or slot G - 1 - c of the odd rounds when
+// `snake` (serpentine: on a longest-first list the CTA that took a round's
+// longest item takes the next round's shortest).  Strictly increasing in k,
+// so a CTA's items end at its first slot past the list.
+__device__ __forceinline__ int cta_slot(int k, int snake) {
+  const int c = (snake && (k & 1)) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  return k * (int)gridDim.x + c;
+}
+
 __global__ void __launch_bounds__(ft::THREADS, 1)
     fine_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, const FineTcArgs a) {
@@ -366,10 +376,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long gs = 0;                 // steps loaded
     int k = 0, q_issued = 0;
     bool ok = true;
-    int item_next = blockIdx.x < a.n_items ? a.worklist[blockIdx.x] : 0;
-    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+    const int slot0 = cta_slot(0, a.snake);
+    int item_next = slot0 < a.n_items ? a.worklist[slot0] : 0;
+    for (int slot = slot0; slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
       const int item = item_next;
-      if (slot + (int)gridDim.x < a.n_items) item_next = a.worklist[slot + gridDim.x];
+      const int slot_next = cta_slot(k + 1, a.snake);
+      if (slot_next < a.n_items) item_next = a.worklist[slot_next];
       const int bh = item / g.P, qd = item % g.P;
       const int qb = k % QBUF;
       // lanes 0, 1: the item's two query tiles (a missing second tile repeats the first; its rows
@@ -458,7 +470,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long c = 0;
     int k = 0;
     bool ok = true;
-    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
       const int qb = k % QBUF;
       if (!mbar_wait_warp(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
       const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
@@ -497,7 +509,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long c = 0;
     int k = 0;
     bool ok = true;
-    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
       bool first = true;
       while (true) {
         const int b = (int)(c & 1);
@@ -535,7 +547,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     // before PV(c) has read it and S never waits for a PV to complete.
     long long cs = 0, cp = 0;         // next S step, next PV step
     int ks_item = 0, kp_item = 0;     // their items (in this CTA's slot order)
-    bool s_first = true, s_done = (int)blockIdx.x >= a.n_items, p_first = true;
+    bool s_first = true, s_done = cta_slot(0, a.snake) >= a.n_items, p_first = true;
     int qb_s = 0;
     uint64_t qd = 0;
     auto issue_s = [&]() -> bool {
@@ -565,12 +577,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       if (meta & STEP_LAST) {
         ++ks_item;
         s_first = true;
-        if ((long long)blockIdx.x + (long long)ks_item * gridDim.x >= a.n_items) s_done = true;
+        if (cta_slot(ks_item, a.snake) >= a.n_items) s_done = true;
       }
       return true;
     };
     bool ok = issue_s() && issue_s();
-    for (int slot = blockIdx.x; ok && slot < a.n_items;) {
+    for (int slot = cta_slot(0, a.snake); ok && slot < a.n_items;) {
       const int b = (int)(cp & 1);
       const int vs = (int)(cp % VST);
       if (p_first && kp_item >= 1 &&
@@ -592,7 +604,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       if (info & STEP_LAST) {
         ++kp_item;
         p_first = true;
-        slot += gridDim.x;
+        slot = cta_slot(kp_item, a.snake);
       }
       ok = issue_s();
     }
@@ -607,7 +619,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long c = 0;
     int k = 0;
     bool ok = true;
-    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
       const int qb = k % QBUF;
       if (!mbar_wait(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
       const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
@@ -654,7 +666,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long c = 0;
     int k = 0;
     bool ok = true;
-    for (int slot = blockIdx.x; slot < a.n_items && ok; slot += gridDim.x, ++k) {
+    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
       bool first = true;
       while (true) {
         const int b = (int)(c & 1);
@@ -704,10 +716,12 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     const float sl2 = g.scale * 1.4426950408889634f;
     long long c = 0;
     int k = 0;
-    int item_next = blockIdx.x < a.n_items ? a.worklist[blockIdx.x] : 0;
-    for (int slot = blockIdx.x; slot < a.n_items; slot += gridDim.x, ++k) {
+    const int slot0 = cta_slot(0, a.snake);
+    int item_next = slot0 < a.n_items ? a.worklist[slot0] : 0;
+    for (int slot = slot0; slot < a.n_items; ++k, slot = cta_slot(k, a.snake)) {
       const int item = item_next;                     // the next item's code loads during this one
-      if (slot + (int)gridDim.x < a.n_items) item_next = a.worklist[slot + gridDim.x];
+      const int slot_next = cta_slot(k + 1, a.snake);
+      if (slot_next < a.n_items) item_next = a.worklist[slot_next];
       const int bh = item / g.P, qd = item % g.P;
       const int tile = kItemTiles * qd + half;
       const bool valid = tile < g.nT;

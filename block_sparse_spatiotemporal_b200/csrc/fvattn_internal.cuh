@@ -106,6 +106,7 @@ struct FineTcArgs {
   const int* ucount;
   const int* worklist;
   int n_items;
+  int snake;             // 1: serpentine slots (the forward's own list); 0: CTA c runs c, c + G, ...
   const int* tile_cube;
   int q_nat, k_nat, v_nat;
   __nv_bfloat16* out;

@@ -198,10 +198,11 @@ int fvattn_pool_select_noalloc_status(fvattn_stream_t stream, int32_t* status);
  * (longest-processing-time first).  worklist has B*H*P int32.  (The work
  * list fvattn_forward and fvattn_block_sparse_fwd build for their own fine
  * stage ranks union sizes in buckets of 16 entries, ties by item, so that
- * items of one head run together, and applies that order within groups of
- * consecutive heads when one head's K and V take more than a quarter of the
- * L2: groups of about 40 MB of K/V, in head order, so that the CTAs running
- * together share those heads' K/V in the cache.) */
+ * items of one head run together, runs it serpentine (CTA c takes slot c of
+ * even rounds of G slots and slot G - 1 - c of odd ones), and applies that
+ * order within groups of consecutive heads when one head's K and V take more
+ * than a quarter of the L2: groups of about 40 MB of K/V, in head order, so
+ * that the CTAs running together share those heads' K/V in the cache.) */
 int fvattn_build_worklist(const fvattn_shape* shape, const fvattn_blocks* blocks,
                           int32_t* worklist, void* ws, size_t ws_bytes, fvattn_stream_t stream);
 
