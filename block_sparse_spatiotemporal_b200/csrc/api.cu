@@ -110,6 +110,7 @@ WsLayout layout_for(const Geom& g, int dtype, const fvattn_rope* r, bool sub = f
   L.qcost = take(sizeof(int) * (size_t)g.BH * g.Qn);
   L.cta_times = take(sizeof(unsigned long long) * (1 + 2 * (size_t)kMaxCtas));
   L.cta_busy = take(sizeof(long long) * (size_t)kMaxCtas);
+  L.next_slot = take(sizeof(int));
   // RoPE: the rotated K (tiled); the rotated Q goes to the caller's output buffer
   L.krot = take(rope_on(r) ? (size_t)g.BH * g.N * g.d * elem_size(dtype) : 0);
   if (sub) {
@@ -445,6 +446,10 @@ int run_coarse(const Call& c, const fvattn_shape* shape, const void* q, const vo
 // (480p: DRAM reads of the fine stage 3.27 -> 2.30 GB a launch, same time),
 // and a bucket's spread is small against the tail the light items fill.
 constexpr int kLptShift = 4;
+#ifndef FVATTN_FT_DYNAMIC
+#define FVATTN_FT_DYNAMIC 1
+#endif
+constexpr bool kFineDynamic = FVATTN_FT_DYNAMIC != 0;
 int heads_per_group(const Geom& g, int dtype) {
   const double per_head = 2.0 * (double)g.N * g.d * elem_size(dtype);
   if (per_head <= 126.0e6 / 4) return g.BH;
@@ -538,9 +543,15 @@ int run_fine(const Call& c, const fvattn_shape* shape, const void* q, const void
     a.ucount = c.at<int>(c.L.ucount);
     a.worklist = worklist ? worklist : c.at<int>(c.L.worklist);
     a.n_items = c.g.BH * c.g.P;
-    // the schedule's own list runs serpentine; a caller's list (the augmentation's
-    // kept work list, whose per-CTA loads assume CTA c runs c, c + G, ...) does not
+    // the schedule's own list is handed out greedily (each CTA takes the next
+    // slot when it starts an item) or serpentine; a caller's list (the
+    // augmentation's kept work list, whose per-CTA loads assume CTA c runs
+    // c, c + G, ...) keeps that static order
     a.snake = worklist ? 0 : 1;
+    if (!worklist && kFineDynamic) {
+      a.next_slot = c.at<int>(c.L.next_slot);
+      FV_CUDA(cudaMemsetAsync(a.next_slot, 0, sizeof(int), c.s));
+    }
     a.tile_cube = c.at<int>(c.L.tile_cube);
     a.q_nat = natural;
     a.k_nat = k_nat;

@@ -51,20 +51,12 @@ namespace ft {
 #ifndef FVATTN_FT_QBUF
 #define FVATTN_FT_QBUF 1
 #endif
-// MMA issue: 0 = lane 0 of warps 1 (S) and 2 (PV); 1 = the same two roles as
-// whole warps with an elected issuing lane; 2 = one warp issues both, PV(c)
-// then S(c + 2), so S never waits for a PV to complete (in-order execution
-// of one thread's tcgen05.mma keeps S(c + 2) from overwriting P(c) early).
-#ifndef FVATTN_FT_ISSUE
-#define FVATTN_FT_ISSUE 0
-#endif
 
 constexpr int D = 128;
 constexpr int KST = FVATTN_FT_KSTAGES;     // K ring depth
 constexpr int VST = FVATTN_FT_VSTAGES;     // V ring depth
 constexpr int QBUF = FVATTN_FT_QBUF;       // Q buffers (items in flight)
 constexpr int SBUF = 2;                    // TMEM S buffers
-constexpr int ISSUE = FVATTN_FT_ISSUE;
 constexpr int THREADS = 384;
 constexpr int SM_WARP0 = 4;                             // first softmax warp
 constexpr uint32_t BOX = 64 * 128;                      // one 64-row x 128-byte box: 8 KB
@@ -77,8 +69,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 256;                        // O of keys 0-31; keys 32-63 at +128
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, false, true);
-constexpr int ENTRY_LAST = 1 << 22;   // union entry word: last entry of the item
 constexpr int STEP_LAST = 1 << 4;     // step word: sel of tile 0 (bits 0-1), tile 1 (bits 2-3), last
+constexpr int STEP_END = 1 << 5;      // step word: the CTA has no further item
+constexpr int kItemRing = 8;          // item codes in flight between the producer and the softmax
 
 struct Ctl {
   uint64_t q_full[QBUF], q_empty[QBUF];
@@ -95,6 +88,8 @@ struct Ctl {
   uint64_t drain;          // final commits of the two MMA threads
   int info[SBUF];          // per S buffer: the step word
   int meta[KST];
+  int item_ring[kItemRing]; // item code of this CTA's k-th item at k % kItemRing (-1: no more items),
+                            // written by the producer before the item's Q arrival
   float2 ex[128];                 // epilogue exchange per row: group 1's (m, l), then the scales
                                   // (s0, s1) group 0 computed from both groups' (m, l)
   uint32_t tmem_base;
@@ -347,7 +342,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     mbar_init(&ctl->o_empty, 8);
     mbar_init(&ctl->xchg1, 4);
     mbar_init(&ctl->xchg2, 4);
-    mbar_init(&ctl->drain, ISSUE == 2 ? 1 : 2);   // one final commit per MMA issuer
+    mbar_init(&ctl->drain, 2);   // one final commit per MMA issuer
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -376,11 +371,20 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     long long gs = 0;                 // steps loaded
     int k = 0, q_issued = 0;
     bool ok = true;
-    const int slot0 = cta_slot(0, a.snake);
-    int item_next = slot0 < a.n_items ? a.worklist[slot0] : 0;
-    for (int slot = slot0; slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
+    // This CTA's items: the work-list slots cta_slot(k), or (a.next_slot) slot
+    // blockIdx.x first and then each slot taken from the shared counter when
+    // the previous item starts (greedy list scheduling, one item ahead).
+    int slot = a.next_slot ? (int)blockIdx.x : cta_slot(0, a.snake);
+    int slot_next = 0;
+    int item_next = slot < a.n_items ? a.worklist[slot] : 0;
+    for (; slot < a.n_items && ok; ++k, slot = slot_next) {
       const int item = item_next;
-      const int slot_next = cta_slot(k + 1, a.snake);
+      if (a.next_slot) {
+        if (leader) slot_next = (int)gridDim.x + atomicAdd(a.next_slot, 1);
+        slot_next = __shfl_sync(0xffffffffu, slot_next, 0);
+      } else {
+        slot_next = cta_slot(k + 1, a.snake);
+      }
       if (slot_next < a.n_items) item_next = a.worklist[slot_next];
       const int bh = item / g.P, qd = item % g.P;
       const int qb = k % QBUF;
@@ -397,6 +401,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
       const int qc0 = __shfl_sync(0xffffffffu, qcube, 0), qc1 = __shfl_sync(0xffffffffu, qcube, 1);
       const int qt0 = __shfl_sync(0xffffffffu, qtile, 0), qt1 = __shfl_sync(0xffffffffu, qtile, 1);
       if (leader) {
+        ctl->item_ring[k % kItemRing] = item;     // released by the arrival below
         mbar_arrive_expect_tx(&ctl->q_full[qb], Q_BYTES);
         uint8_t* qd_smem = sQ + qb * Q_BYTES;
         tma_tile(&mq, a.q_nat, qc0, bh, qt0, qd_smem, Q_HALF, &ctl->q_full[qb]);
@@ -465,163 +470,38 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         mbar_drain(&ctl->v_full[i], (uint32_t)(last / VST) & 1, a.status, cap);
       }
     }
-  } else if (ISSUE == 1 && warp == 1) {
-    // ------------------------------------------- MMA: S (whole warp, elected lane)
-    long long c = 0;
-    int k = 0;
-    bool ok = true;
-    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
+    // then the end of this CTA's items: a Q buffer that carries no rows,
+    // item code -1 (after the drain above, which waits for the last loaded
+    // phase of each Q buffer)
+    if (ok) {
       const int qb = k % QBUF;
-      if (!mbar_wait_warp(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
-      const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
-      while (true) {
-        const int ks = (int)(c % KST);
-        const int b = (int)(c & 1);
-        if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(c / KST) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        if (c >= SBUF &&
-            !mbar_wait_warp(&ctl->pv_done[b], (uint32_t)((c - SBUF) >> 1) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        const int meta = ctl->meta[ks];
-        tc_fence_after();
-        if (elect_one()) {
-          ctl->info[b] = meta;
-          s_mmas(tbase + 128 * b, qd, umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024));
-          mma_commit(&ctl->s_full[b]);
-          mma_commit(&ctl->k_empty[ks]);
-          if (meta & STEP_LAST) mma_commit(&ctl->q_empty[qb]);
-          mbar_arrive(&ctl->s_full[b]);
-        }
-        __syncwarp();
-        ++c;
-        if (meta & STEP_LAST) break;
+      if (leader && k >= QBUF) ok = mbar_wait(&ctl->q_empty[qb], ((k / QBUF) - 1) & 1, abort_flag, a.status, cap);
+      if (leader && ok) {
+        ctl->item_ring[k % kItemRing] = -1;
+        mbar_arrive(&ctl->q_full[qb]);
       }
     }
-    if (elect_one()) mma_commit(&ctl->drain);
-    __syncwarp();
-    mbar_drain(&ctl->drain, 0, a.status, cap);
-  } else if (ISSUE == 1 && warp == 2) {
-    // ------------------------------------------ MMA: PV (whole warp, elected lane)
-    long long c = 0;
-    int k = 0;
-    bool ok = true;
-    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
-      bool first = true;
-      while (true) {
-        const int b = (int)(c & 1);
-        const int vs = (int)(c % VST);
-        if (first && k >= 1 && !mbar_wait_warp(&ctl->o_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait_warp(&ctl->v_full[vs], (uint32_t)(c / VST) & 1, abort_flag, a.status, cap) ||
-            !mbar_wait_warp(&ctl->p_full[b], (uint32_t)(c >> 1) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        const int info = ctl->info[b];
-        tc_fence_after();
-        if (elect_one()) {
-          pv_mmas(tbase, tbase + 128 * b, sV + vs * STAGE_BYTES, first);
-          mma_commit(&ctl->pv_done[b]);
-          mma_commit(&ctl->v_empty[vs]);
-        }
-        __syncwarp();
-        first = false;
-        ++c;
-        if (info & STEP_LAST) break;
-      }
-    }
-    if (elect_one()) mma_commit(&ctl->drain);
-    __syncwarp();
-    mbar_drain(&ctl->drain, 0, a.status, cap);
-  } else if (ISSUE == 2 && warp == 1) {
-    // ------------------------------------ MMA: S and PV from one warp, in order
-    // Order of issue: S(0), S(1), then per step c: PV(c) once P(c) is
-    // written, then S(c + 2) into the buffer PV(c) reads.  One thread's
-    // tcgen05.mma run in issue order, so S(c + 2) cannot overwrite P(c)
-    // before PV(c) has read it and S never waits for a PV to complete.
-    long long cs = 0, cp = 0;         // next S step, next PV step
-    int ks_item = 0, kp_item = 0;     // their items (in this CTA's slot order)
-    bool s_first = true, s_done = cta_slot(0, a.snake) >= a.n_items, p_first = true;
-    int qb_s = 0;
-    uint64_t qd = 0;
-    auto issue_s = [&]() -> bool {
-      if (s_done) return true;
-      if (s_first) {
-        qb_s = ks_item % QBUF;
-        if (!mbar_wait_warp(&ctl->q_full[qb_s], (uint32_t)(ks_item / QBUF) & 1, abort_flag, a.status, cap))
-          return false;
-        qd = umma_desc_sw128(smem_u32(sQ + qb_s * Q_BYTES), 16, 1024);
-        s_first = false;
-      }
-      const int ks = (int)(cs % KST);
-      const int b = (int)(cs & 1);
-      if (!mbar_wait_warp(&ctl->k_full[ks], (uint32_t)(cs / KST) & 1, abort_flag, a.status, cap)) return false;
-      const int meta = ctl->meta[ks];
-      tc_fence_after();
-      if (elect_one()) {
-        ctl->info[b] = meta;
-        s_mmas(tbase + 128 * b, qd, umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024));
-        mma_commit(&ctl->s_full[b]);
-        mma_commit(&ctl->k_empty[ks]);
-        if (meta & STEP_LAST) mma_commit(&ctl->q_empty[qb_s]);
-        mbar_arrive(&ctl->s_full[b]);
-      }
-      __syncwarp();
-      ++cs;
-      if (meta & STEP_LAST) {
-        ++ks_item;
-        s_first = true;
-        if (cta_slot(ks_item, a.snake) >= a.n_items) s_done = true;
-      }
-      return true;
-    };
-    bool ok = issue_s() && issue_s();
-    for (int slot = cta_slot(0, a.snake); ok && slot < a.n_items;) {
-      const int b = (int)(cp & 1);
-      const int vs = (int)(cp % VST);
-      if (p_first && kp_item >= 1 &&
-          !mbar_wait_warp(&ctl->o_empty, (uint32_t)(kp_item - 1) & 1, abort_flag, a.status, cap))
-        break;
-      if (!mbar_wait_warp(&ctl->v_full[vs], (uint32_t)(cp / VST) & 1, abort_flag, a.status, cap) ||
-          !mbar_wait_warp(&ctl->p_full[b], (uint32_t)(cp >> 1) & 1, abort_flag, a.status, cap))
-        break;
-      const int info = ctl->info[b];
-      tc_fence_after();
-      if (elect_one()) {
-        pv_mmas(tbase, tbase + 128 * b, sV + vs * STAGE_BYTES, p_first);
-        mma_commit(&ctl->pv_done[b]);
-        mma_commit(&ctl->v_empty[vs]);
-      }
-      __syncwarp();
-      p_first = false;
-      ++cp;
-      if (info & STEP_LAST) {
-        ++kp_item;
-        p_first = true;
-        slot = cta_slot(kp_item, a.snake);
-      }
-      ok = issue_s();
-    }
-    if (elect_one()) mma_commit(&ctl->drain);
-    __syncwarp();
-    mbar_drain(&ctl->drain, 0, a.status, cap);
-  } else if (ISSUE == 0 && warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------- MMA: S
     // S(c) into buffer c & 1 once the PV of step c - 2, which read its P
     // from that buffer, is complete; a K stage is released when its S
-    // completes, the Q buffer after the item's last S.
+    // completes, the Q buffer after the item's last S.  The producer ends
+    // the CTA's items with a Q buffer that carries no rows (item code -1 in
+    // the ring): passed on to the softmax as a step word with STEP_END.
     long long c = 0;
-    int k = 0;
     bool ok = true;
-    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
+    for (int k = 0; ok; ++k) {
       const int qb = k % QBUF;
       if (!mbar_wait(&ctl->q_full[qb], (uint32_t)(k / QBUF) & 1, abort_flag, a.status, cap)) break;
+      if (ctl->item_ring[k % kItemRing] < 0) {
+        const int b = (int)(c & 1);
+        if (c >= SBUF && !mbar_wait(&ctl->pv_done[b], (uint32_t)((c - SBUF) >> 1) & 1, abort_flag, a.status, cap))
+          break;
+        ctl->info[b] = STEP_END;
+        mbar_arrive(&ctl->s_full[b]);     // both arrivals of the buffer's phase, no MMA
+        mbar_arrive(&ctl->s_full[b]);
+        break;
+      }
       const uint64_t qd = umma_desc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
       while (true) {
         const int ks = (int)(c % KST);
@@ -638,13 +518,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         const int meta = ctl->meta[ks];
         ctl->info[b] = meta;
         tc_fence_after();
-        const uint64_t kd = umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024);
-        const uint32_t tS = tbase + 128 * b;
-        mma_ss(tS, qd, kd, IDESC_S, 0u);
-#pragma unroll
-        for (int kk = 1; kk < 8; ++kk)
-          mma_ss(tS, qd + (((kk >> 2) * Q_HALF + (kk & 3) * 32) >> 4),
-                 kd + (((kk >> 2) * K_HALF + (kk & 3) * 32) >> 4), IDESC_S, 1u);
+        s_mmas(tbase + 128 * b, qd, umma_desc_sw128(smem_u32(sK + ks * STAGE_BYTES), 16, 1024));
         mma_commit(&ctl->s_full[b]);
         mma_commit(&ctl->k_empty[ks]);
         mbar_arrive(&ctl->s_full[b]);
@@ -657,26 +531,22 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     // every MMA this thread issued has completed before TMEM is freed
     mma_commit(&ctl->drain);
     mbar_drain(&ctl->drain, 0, a.status, cap);
-  } else if (ISSUE == 0 && warp == 2 && lane == 0) {
+  } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------------ MMA: PV
     // O_t += P_t V_t for the step's key tiles t = 0, 1 once both softmax
     // groups wrote P; the first step of an item overwrites O after the
     // previous item's epilogue read it.  A V stage is released when its PV
-    // completes.
+    // completes.  A step word with STEP_END (no V loaded for it) ends the loop.
     long long c = 0;
-    int k = 0;
     bool ok = true;
-    for (int slot = cta_slot(0, a.snake); slot < a.n_items && ok; ++k, slot = cta_slot(k, a.snake)) {
+    bool end = false;
+    for (int k = 0; ok && !end; ++k) {
       bool first = true;
       while (true) {
         const int b = (int)(c & 1);
         const int vs = (int)(c % VST);
-        // O free and V loaded come well before P, the wait on the critical path
+        // O free comes well before P, the wait on the critical path
         if (first && k >= 1 && !mbar_wait(&ctl->o_empty, (uint32_t)(k - 1) & 1, abort_flag, a.status, cap)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(&ctl->v_full[vs], (uint32_t)(c / VST) & 1, abort_flag, a.status, cap)) {
           ok = false;
           break;
         }
@@ -685,17 +555,16 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
           break;
         }
         const int info = ctl->info[b];
-        tc_fence_after();
-        const uint32_t tP = tbase + 128 * b;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const uint64_t vd = umma_desc_sw128(smem_u32(sV + vs * STAGE_BYTES + t * V_TILE), BOX, 1024);
-          const uint32_t tO = tbase + TMEM_O + 128 * t;
-          // 16 keys = 16 V rows = 2048 bytes per K step; P of tile t in columns 64 t .. 64 t + 31
-          mma_ts(tO, tP + 64 * t, vd, IDESC_PV, first ? 0u : 1u);
-#pragma unroll
-          for (int kk = 1; kk < 4; ++kk) mma_ts(tO, tP + 64 * t + 8 * kk, vd + ((kk * 2048) >> 4), IDESC_PV, 1u);
+        if (info & STEP_END) {
+          end = true;
+          break;
         }
+        if (!mbar_wait(&ctl->v_full[vs], (uint32_t)(c / VST) & 1, abort_flag, a.status, cap)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv_mmas(tbase, tbase + 128 * b, sV + vs * STAGE_BYTES, first);
         mma_commit(&ctl->pv_done[b]);
         mma_commit(&ctl->v_empty[vs]);
         first = false;
@@ -715,17 +584,10 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
     const uint32_t tO = tbase + TMEM_O + 128 * h + lane_off;
     const float sl2 = g.scale * 1.4426950408889634f;
     long long c = 0;
-    int k = 0;
-    const int slot0 = cta_slot(0, a.snake);
-    int item_next = slot0 < a.n_items ? a.worklist[slot0] : 0;
-    for (int slot = slot0; slot < a.n_items; ++k, slot = cta_slot(k, a.snake)) {
-      const int item = item_next;                     // the next item's code loads during this one
-      const int slot_next = cta_slot(k + 1, a.snake);
-      if (slot_next < a.n_items) item_next = a.worklist[slot_next];
-      const int bh = item / g.P, qd = item % g.P;
-      const int tile = kItemTiles * qd + half;
-      const bool valid = tile < g.nT;
-      const int cube = valid && a.out_nat ? a.tile_cube[tile] : 0;   // used by the epilogue
+    bool end = false;
+    for (int k = 0; !end; ++k) {
+      int bh = 0, qd = 0, tile = 0, cube = 0;         // the item's, read at its first step
+      bool valid = false, first = true;
       float m_use = -INFINITY, l = 0.f;
       bool ok = true;
       while (true) {
@@ -736,6 +598,21 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         }
         tc_fence_after();
         const int info = ctl->info[b];
+        if (info & STEP_END) {                        // no further item; the PV thread stops on it too
+          mbar_arrive_warp(&ctl->p_full[b]);
+          end = true;
+          break;
+        }
+        if (first) {
+          // the item's code, written by the producer before its Q arrival
+          const int item = ctl->item_ring[k % kItemRing];
+          bh = item / g.P;
+          qd = item % g.P;
+          tile = kItemTiles * qd + half;
+          valid = tile < g.nT;
+          cube = valid && a.out_nat ? a.tile_cube[tile] : 0;   // used by the epilogue
+          first = false;
+        }
         const bool sel = (info >> (2 * h + half)) & 1;
         const uint32_t tS = tbase + 128 * b + 64 * h + lane_off;
         uint32_t pk[32];
@@ -787,7 +664,7 @@ __global__ void __launch_bounds__(ft::THREADS, 1)
         ++c;
         if (info & STEP_LAST) break;
       }
-      if (!ok) break;
+      if (!ok || end) break;
       // ---- epilogue: merge the groups' (m, l, O); this group writes dims 64 h .. 64 h + 63
       if (!mbar_wait(&ctl->pv_done[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1, abort_flag, a.status, cap)) break;
       tc_fence_after();

@@ -66,6 +66,7 @@ struct WsLayout {
   size_t useg, qcost;    // int32 [BH*Qn] quad items: union segments and cost
   size_t cta_times;      // u64 [1 + 2 * kMaxCtas] fine-stage CTA start / end times (profiling)
   size_t cta_busy;       // i64 [kMaxCtas] measured CTA busy times for the augmentation's slack
+  size_t next_slot;      // int32 work-list counter of the fine stage's greedy dispatch
   size_t rank;           // int32 [BH*P] scratch of the work-list sort
   size_t krot;           // dtype [BH*N*d] rotated K, tiled (rope only)
   size_t sqh, sql;       // sub-block scoring only: float [BH*nT*8*d] pooled sub-blocks of Q (tf32 hi + lo)
@@ -107,6 +108,8 @@ struct FineTcArgs {
   const int* worklist;
   int n_items;
   int snake;             // 1: serpentine slots (the forward's own list); 0: CTA c runs c, c + G, ...
+  int* next_slot;        // optional: zeroed counter; CTA c starts with slot c and then takes
+                         // slot G + atomicAdd(next_slot, 1) when it starts an item (greedy)
   const int* tile_cube;
   int q_nat, k_nat, v_nat;
   __nv_bfloat16* out;
