@@ -5,9 +5,13 @@
 // Persistent kernel, one CTA per SM, 384 threads.  A work item is two
 // adjacent query tiles of one head: one 128-row tensor-core tile walking the
 // union of the two tiles' key lists two entries (128 keys) per step.
-//   warp 0       TMA producer: the item's Q, K of every step's two key
-//                tiles into a 2-stage ring and V into a 3-stage ring (V is
-//                consumed last, so its ring is the deeper one);
+//   warp 0       TMA producer: picks the CTA's next item (the next slot of
+//                a work-list counter when it starts an item, or a static
+//                slot sequence) and publishes its code in a shared ring;
+//                loads the item's Q, K of every step's two key tiles into a
+//                3-stage ring and V into a 3-stage ring; after the last item
+//                it arrives on the next Q buffer without rows (code -1),
+//                which every role passes on and stops at;
 //   warp 1       S issuer (one thread): S = Q K^T (M=128, N=128, K=128) of
 //                step c into TMEM S buffer c & 1 once the PV of step c - 2
 //                (the buffer's previous P) is complete;
@@ -35,7 +39,7 @@
 // key tile 0 at [256, 384), of key tile 1 at [384, 512), fp32.
 // Shared memory (1024-aligned, 128-byte swizzle), default build:
 //   Q    = 2 d-halves x 128 rows x 128 B                    32 KB
-//   K[2] = 2 x (2 d-halves x 128 keys x 128 B)              64 KB
+//   K[3] = 3 x (2 d-halves x 128 keys x 128 B)              96 KB
 //   V[3] = 3 x (2 tiles x 2 d-halves x 64 keys x 128 B)     96 KB
 #include "fvattn_internal.cuh"
 
